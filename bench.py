@@ -1,0 +1,318 @@
+"""Benchmark: exact attention forward + backward on B200, TFLOPS and fraction of peak.
+
+One step = the whole hot path once over one batch: fa_fwd then fa_bwd (row-sum
+preprocess, dK/dV/dQ kernel, dQ conversion) on the shape
+B=2, S=16384, H=16 (Hq = Hkv), d=128, non-causal, bf16, inputs N(0, 1) -- the shape
+shared by the d=128 forward sweep (batch = 32768 / seqlen at 16k) and the backward
+configuration (B=2, 16k).  FLOPs follow the metric's definition: forward
+4*B*Hq*Sq*Sk*d (halved for causal), backward 2.5x that.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (weak scaling, independent replicas): torchrun ... bench.py --gpus N
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(B=2, S=16384, H=16, d=128, causal=False)
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def flops(B, Sq, Sk, H, d, causal):
+    f = 4.0 * B * H * Sq * Sk * d
+    if causal:
+        f /= 2.0
+    return f, 2.5 * f
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_cpu_baseline(budget_s=15.0):
+    """Time the fp64 oracle on a bounded sample of the workload: full-length query rows
+    of one head through the forward (O, LSE) and the backward dQ path.  Returns the
+    oracle's rate in the metric's unit (algorithmic TFLOPS for those rows)."""
+    import oracle
+    from exact_attention_blackwell_fa_b200.inputs import Shape, make_inputs
+
+    W = WORKLOAD
+    # one (batch, head) slice at full sequence length stands in for the workload
+    shape = Shape(1, W["S"], W["S"], 1, 1, W["d"])
+    q, k, v, do = make_inputs(shape, seed=0, with_dout=True)
+    nrows = 8
+    done_rows = 0
+    t0 = time.perf_counter()
+    while True:
+        rows = torch.tensor([[0, 0, (done_rows + i) % W["S"]] for i in range(nrows)])
+        oracle.fwd(q, k, v, causal=W["causal"], rows=rows)
+        oracle.bwd(q, k, v, do, causal=W["causal"], qrows=rows)
+        done_rows += nrows
+        if time.perf_counter() - t0 > budget_s:
+            break
+    el = time.perf_counter() - t0
+    per_row = 4.0 * W["S"] * W["d"] * (1.0 + 2.5)
+    return {"value": done_rows * per_row / el / 1e12, "unit": "TFLOPS",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{done_rows} full-length query rows (Sk={W['S']}, d={W['d']}) of one "
+                      f"head through forward + backward-dQ, fp64, {el:.1f} s"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fwd-only", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    W = WORKLOAD
+    f_fwd, f_bwd = flops(W["B"], W["S"], W["S"], W["H"], W["d"], W["causal"])
+    config = {"workload": f"attention fwd+bwd bf16 B={W['B']} S={W['S']} H={W['H']} "
+                          f"d={W['d']} {'causal' if W['causal'] else 'non-causal'}",
+              "B": W["B"], "seq_len": W["S"], "heads": W["H"], "head_dim": W["d"],
+              "causal": W["causal"], "global_batch": W["B"] * world,
+              "parallelism": f"replicas x{world} (independent batches, no collective)",
+              "l2": "inputs larger than L2 (each of Q, K, V, O, dO is 128 MiB)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        # The reference arm is the fp64 oracle on the host cores (no GPU code).
+        steps = []
+        for _ in range(args.warmup):
+            pass
+        cb = None
+        for _ in range(max(1, args.steps)):
+            cb = oracle_cpu_baseline(budget_s=max(2.0, 60.0 / max(1, args.steps)))
+            steps.append(cb["value"])
+        val = statistics.median(steps)
+        print(json.dumps({
+            "impl": "reference", "metric": "attention fwd+bwd TFLOPS (fp64 oracle on host cores)",
+            "value": val, "unit": "TFLOPS", "n_gpus": 0, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "dtype": "f64",
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {**cb, "value": val},
+            "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return
+
+    import exact_attention_blackwell_fa_b200 as fa
+    from exact_attention_blackwell_fa_b200.inputs import Shape, make_inputs
+
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+
+    shape = Shape(W["B"], W["S"], W["S"], W["H"], W["H"], W["d"])
+    q, k, v, do = make_inputs(shape, seed=rank, device=dev, with_dout=True)
+    do_bwd = not args.fwd_only
+    o = torch.empty_like(q)
+    lse = torch.empty(W["B"], W["H"], W["S"], dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_size(W["B"], W["S"], W["H"], W["d"]), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fa_fwd(q, k, v, causal=W["causal"], out=o, lse=lse, stream=stream)
+        if do_bwd:
+            fa.fa_bwd(q, k, v, o, lse, do, causal=W["causal"], dq=dq, dk=dk, dv=dv,
+                      workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    code, detail = fa.fa_last_device_status(stream)
+    if code != 0:
+        raise RuntimeError(f"device status {code} detail {detail:#x} after warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        fa.fa_fwd(q, k, v, causal=W["causal"], out=o, lse=lse, stream=stream)
+        ev[i][1].record(stream)
+        if do_bwd:
+            fa.fa_bwd(q, k, v, o, lse, do, causal=W["causal"], dq=dq, dk=dk, dv=dv,
+                      workspace=ws, stream=stream)
+        ev[i][2].record(stream)
+    end.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) if do_bwd else 0.0
+    ms_per_step = total_ms / K
+    step_flops = f_fwd + (f_bwd if do_bwd else 0.0)
+    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+    code, detail = fa.fa_last_device_status(stream)
+    if code != 0:
+        raise RuntimeError(f"device status {code} detail {detail:#x} after timing")
+
+    # end-to-end through the public API with host buffers: pinned H2D of the step's
+    # inputs, the step, D2H of its outputs, all inside the timed region
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+    ho, hdq, hdk, hdv = (torch.empty_like(t, device="cpu").pin_memory() for t in (o, dq, dk, dv))
+    hlse = torch.empty_like(lse, device="cpu").pin_memory()
+    E = max(3, K // 4)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        if do_bwd:
+            do.copy_(hdo, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+        if do_bwd:
+            hdq.copy_(dq, non_blocking=True)
+            hdk.copy_(dk, non_blocking=True)
+            hdv.copy_(dv, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / E
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    nbytes = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
+    h2d = nbytes(q, k, v) + (nbytes(do) if do_bwd else 0)
+    d2h = nbytes(o, lse) + (nbytes(dq, dk, dv) if do_bwd else 0)
+
+    peaks, peak_kind = load_peaks()
+    # dominant kernel: the backward's dK/dV/dQ kernel when the backward runs, else the
+    # forward kernel; its per-launch time is the CUDA-event time of its call
+    if do_bwd and bwd_ms > fwd_ms:
+        dom, dom_ms, dom_flops = "fa_bwd (dkdv + preprocess + convert)", bwd_ms, f_bwd
+    else:
+        dom, dom_ms, dom_flops = "fa_fwd_kernel", fwd_ms, f_fwd
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    out = {
+        "metric": "attention fwd/bwd TFLOPS at 1 B200 and fraction of 2.25 PFLOPS BF16 peak",
+        "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config,
+        "frac_of_2250": value / world / NOMINAL_BF16_TFLOPS,
+        "fwd": {"ms": fwd_ms, "tflops": f_fwd / (fwd_ms * 1e-3) / 1e12,
+                "frac_of_2250": f_fwd / (fwd_ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS},
+        "bwd": ({"ms": bwd_ms, "tflops": f_bwd / (bwd_ms * 1e-3) / 1e12,
+                 "frac_of_2250": f_bwd / (bwd_ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS}
+                if do_bwd else None),
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                     "peak_kind": f"{peak_kind} sustained bf16 (cuBLAS loop)",
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None},
+        "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * (1 + (3 if do_bwd else 0)),
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = oracle_cpu_baseline()
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

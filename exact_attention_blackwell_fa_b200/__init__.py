@@ -1,1 +1,137 @@
-"""Exact scaled-dot-product attention (forward and backward) for B200 / sm_100a."""
+"""Exact scaled-dot-product attention (forward and backward) for B200 / sm_100a.
+
+Thin Python binding over the C ABI in include/fa.h (libfa.so).  PyTorch supplies
+device memory and the current stream; every step of the computation runs in the
+library's CUDA kernels.  The functions carry the C names:
+
+    fa_fwd(q, k, v, causal=False, scale=None) -> (o, lse)
+    fa_bwd(q, k, v, o, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
+    fa_bwd_workspace_size(B, Sq, Hq, d) -> int
+    fa_status_string(code) -> str
+    fa_last_device_status() -> (code, detail)
+    fa_clear_device_status()
+    fa_debug_inject(mode)
+
+Tensors are CUDA, contiguous, [batch, seq, heads, head_dim], bf16 or fp16; LSE is
+float32 [batch, Hq, Sq].  A non-OK status raises FAError; nothing falls back.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+
+__all__ = [
+    "FAError", "fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_status_string",
+    "fa_last_device_status", "fa_clear_device_status", "fa_debug_inject",
+]
+
+
+class FAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {fa_status_string(code)}")
+
+
+def fa_status_string(code: int) -> str:
+    return _lib.load().fa_status_string(int(code)).decode()
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return _lib.FA_BF16
+    if t.dtype == torch.float16:
+        return _lib.FA_FP16
+    raise TypeError(f"fa: inputs must be bf16 or fp16, got {t.dtype}")
+
+
+def _check(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"fa: {name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"fa: {name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"fa: {name} has dtype {t.dtype}, expected {dtype}")
+
+
+def _raise(code: int, where: str):
+    if code != _lib.FA_OK:
+        raise FAError(code, where)
+
+
+def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+           stream=None):
+    """Forward. q [B,Sq,Hq,d], k/v [B,Sk,Hkv,d] -> (o [B,Sq,Hq,d], lse [B,Hq,Sq] fp32)."""
+    _check(q, "q")
+    _check(k, "k", q.dtype)
+    _check(v, "v", q.dtype)
+    B, Sq, Hq, d = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if k.shape != v.shape or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("fa: k and v must be [B, Sk, Hkv, d] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device=q.device)
+    _check(out, "out", q.dtype)
+    _check(lse, "lse", torch.float32)
+    code = _lib.load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                              lse.data_ptr(), B, Sq, Sk, Hq, Hkv, d, int(bool(causal)),
+                              float(scale), _dtype_code(q), _stream_ptr(stream))
+    _raise(code, "fa_fwd")
+    return out, lse
+
+
+def fa_bwd_workspace_size(B: int, Sq: int, Hq: int, d: int) -> int:
+    return int(_lib.load().fa_bwd_workspace_size(B, Sq, Hq, d))
+
+
+def fa_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+           dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Backward. Returns (dq, dk, dv) in the input dtype."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check(t, name, q.dtype)
+    _check(lse, "lse", torch.float32)
+    B, Sq, Hq, d = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws_bytes = fa_bwd_workspace_size(B, Sq, Hq, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    code = _lib.load().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), B, Sq, Sk, Hq, Hkv, d, int(bool(causal)),
+                              float(scale), _dtype_code(q), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _raise(code, "fa_bwd")
+    return dq, dk, dv
+
+
+def fa_last_device_status(stream=None):
+    """(code, detail) of the device status word; synchronises the stream."""
+    detail = ctypes.c_uint32(0)
+    code = _lib.load().fa_last_device_status(_stream_ptr(stream), ctypes.byref(detail))
+    return int(code), int(detail.value)
+
+
+def fa_clear_device_status(stream=None):
+    _raise(_lib.load().fa_clear_device_status(_stream_ptr(stream)), "fa_clear_device_status")
+
+
+def fa_debug_inject(mode: int):
+    _raise(_lib.load().fa_debug_inject(int(mode)), "fa_debug_inject")

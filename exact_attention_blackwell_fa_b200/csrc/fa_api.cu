@@ -1,0 +1,254 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument validation, TMA tensor
+// maps, device checks and kernel launches.  Every entry point validates first and
+// launches nothing on an invalid argument; there is no alternative code path.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 4-D map over a [B, S, H, d] 16-bit tensor; one box = 64 head-dim columns x 128 rows
+// of one (batch, head), 128-byte swizzled.  Rows past S read as zero.
+bool make_tmap(CUtensorMap* m, const void* ptr, int B, int S, int H, int d, bool bf16)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
+                                   (cuuint64_t)S * H * d * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+               const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+    int sm_count = 0;
+    bool ok = false;  // compute capability 10.0 (B200 class, sm_100a code runs)
+};
+
+constexpr int kMaxDevices = 64;
+
+fa_status device_info(DeviceInfo* out)
+{
+    static DeviceInfo cache[kMaxDevices];
+    static std::mutex mu;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev].sm_count == 0) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FA_ERR_CUDA;
+        cache[dev].sm_count = sms;
+        cache[dev].ok = (major == 10 && minor == 0);
+    }
+    *out = cache[dev];
+    return out->ok ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_common(int B, int Sq, int Sk, int Hq, int Hkv, int d, float scale, fa_dtype dt)
+{
+    if (B < 1 || Sq < 1 || Sk < 1 || Hq < 1 || Hkv < 1) return FA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
+    if (d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+    if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_UNSUPPORTED;
+    // element counts must stay inside the 32-bit row indices the kernels use
+    const long long rows_q = (long long)B * Sq * Hq, rows_k = (long long)B * Sk * Hkv;
+    if (rows_q >= (1LL << 31) || rows_k >= (1LL << 31)) return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+
+int chunk_heads_for(int B, int Hq, int group, int Sk, int d)
+{
+    // heads whose K and V together stay well inside the 126-MB L2
+    const double kv_bytes = 2.0 * Sk * d * 2.0 / group;
+    const double budget = 48.0 * 1024 * 1024;
+    int c = static_cast<int>(budget / (kv_bytes > 1.0 ? kv_bytes : 1.0));
+    if (c < 1) c = 1;
+    if (c > B * Hq) c = B * Hq;
+    return c;
+}
+
+template <typename K>
+fa_status set_smem(K kernel, uint32_t bytes)
+{
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(bytes)) == cudaSuccess
+               ? FA_OK
+               : FA_ERR_CUDA;
+}
+
+int g_inject = 0;
+std::mutex g_inject_mu;
+
+int take_inject()
+{
+    std::lock_guard<std::mutex> lk(g_inject_mu);
+    int v = g_inject;
+    g_inject = 0;
+    return v;
+}
+
+template <int D, bool BF16>
+fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     fa::FwdParams p, int sm_count, cudaStream_t stream)
+{
+    using C = fa::FwdCfg<D, BF16>;
+    fa_status st = set_smem(fa::fa_fwd_kernel<D, BF16>, C::SMEM_BYTES);
+    if (st != FA_OK) return st;
+    const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
+    fa::fa_fwd_kernel<D, BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
+                 int Sk, int Hq, int Hkv, int d, int causal, float scale, fa_dtype dt,
+                 fa_stream stream)
+{
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    fa_status st = check_common(B, Sq, Sk, Hq, Hkv, d, scale, dt);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    DeviceInfo di;
+    st = device_info(&di);
+    if (st != FA_OK) return st;
+    const bool bf16 = dt == FA_BF16;
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap(&tq, q, B, Sq, Hq, d, bf16) || !make_tmap(&tk, k, B, Sk, Hkv, d, bf16) ||
+        !make_tmap(&tv, v, B, Sk, Hkv, d, bf16))
+        return FA_ERR_CUDA;
+    fa::FwdParams p{};
+    p.o = o;
+    p.lse = lse;
+    p.B = B;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.group = Hq / Hkv;
+    const int unit = d == 128 ? 256 : 128;
+    p.num_m = (Sq + unit - 1) / unit;
+    p.num_tiles = B * Hq * p.num_m;
+    p.chunk_heads = chunk_heads_for(B, Hq, p.group, Sk, d);
+    p.causal = causal ? 1 : 0;
+    p.inject = take_inject();
+    p.sl2 = scale * 1.4426950408889634f;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128)
+        return bf16 ? launch_fwd<128, true>(tq, tk, tv, p, di.sm_count, s)
+                    : launch_fwd<128, false>(tq, tk, tv, p, di.sm_count, s);
+    return bf16 ? launch_fwd<256, true>(tq, tk, tv, p, di.sm_count, s)
+                : launch_fwd<256, false>(tq, tk, tv, p, di.sm_count, s);
+}
+
+size_t fa_bwd_workspace_size(int B, int Sq, int Hq, int d)
+{
+    if (B < 1 || Sq < 1 || Hq < 1 || d < 1) return 0;
+    return fa::bwd_workspace_bytes(B, Sq, Hq, d);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq,
+                 int Hkv, int d, int causal, float scale, fa_dtype dt, void* workspace,
+                 size_t workspace_bytes, fa_stream stream)
+{
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+        return FA_ERR_INVALID_ARG;
+    fa_status st = check_common(B, Sq, Sk, Hq, Hkv, d, scale, dt);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return FA_ERR_INVALID_ARG;
+    if (workspace_bytes < fa::bwd_workspace_bytes(B, Sq, Hq, d)) return FA_ERR_INVALID_ARG;
+    DeviceInfo di;
+    st = device_info(&di);
+    if (st != FA_OK) return st;
+    return fa::launch_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Sq, Sk, Hq, Hkv, d, causal != 0,
+                          scale, dt == FA_BF16, workspace, di.sm_count,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+const char* fa_status_string(fa_status s)
+{
+    switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid size, pointer, alignment or scale";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: head_dim, dtype or GPU not supported";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
+    }
+    return "unknown fa_status";
+}
+
+fa_status fa_last_device_status(fa_stream stream, uint32_t* detail)
+{
+    uint32_t h[4] = {0, 0, 0, 0};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyFromSymbolAsync(h, fa::g_status, sizeof(h), 0, cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if (detail) *detail = h[1];
+    return static_cast<fa_status>(h[0]);
+}
+
+fa_status fa_clear_device_status(fa_stream stream)
+{
+    static const uint32_t zero[4] = {0, 0, 0, 0};
+    return cudaMemcpyToSymbolAsync(fa::g_status, zero, sizeof(zero), 0, cudaMemcpyHostToDevice,
+                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? FA_OK
+               : FA_ERR_CUDA;
+}
+
+fa_status fa_debug_inject(int mode)
+{
+    if (mode != 0 && mode != 1) return FA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_inject_mu);
+    g_inject = mode;
+    return FA_OK;
+}
+
+}  // extern "C"

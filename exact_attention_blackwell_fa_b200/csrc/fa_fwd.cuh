@@ -1,0 +1,596 @@
+// fa_fwd.cuh -- exact attention forward for sm_100a.
+//
+// O = softmax(scale Q K^T [+ causal]) V and LSE, tile by tile with an online softmax
+// so the score matrix never reaches HBM ("FlashAttention 4: Snellere,
+// Geheugenefficiente Aandacht voor LLM's", sections "Wat is nieuw in FlashAttention
+// 4", "Software-exponentials via CUDA-kernen", "Slimmere Online
+// Softmax-herwaardering").  The warp roles follow the stages listed there (load,
+// matrix multiply, softmax/normalise, rescale, store); the kernel design is ours:
+//
+//   * persistent CTAs (one per SM) walk a static list of work units
+//     (batch, query head, block of query rows); units are grouped by heads so that the
+//     CTAs running at the same time share K/V through L2, and for the causal mask the
+//     longest units (last query blocks) go first;
+//   * one TMA warp stages Q once per unit and streams K and V through a 5-deep ring
+//     of 32-KB shared-memory chunks (128 rows x 128 head-dim columns, 128-byte
+//     swizzle) guarded by full/empty mbarriers;
+//   * one thread issues tcgen05.mma: S = Q K^T into TMEM, then O += P V with P read
+//     back from TMEM (P overwrites the first half of its own S buffer as 16-bit
+//     pairs);
+//   * softmax warpgroups (thread = query row) load S from TMEM, apply the scale and
+//     mask, keep the running row max / sum, rescale O in TMEM only when the row max
+//     grew by more than kRescaleTau (log2 units), compute P with exp2 split between
+//     the SFU and an FMA-pipe cubic, and finally normalise O and write O and LSE.
+//
+// head_dim 128: two Q tiles (256 query rows) per unit, TMEM = S0 | S1 | O0 | O1; the
+// tensor core alternates between the two tiles so that one tile's softmax overlaps
+// the other tile's MMAs.  head_dim 256: one Q tile, TMEM = S(a) | S(b) | O (256
+// columns); S is double buffered so the next S = Q K^T runs during the softmax.
+#pragma once
+
+#include <type_traits>
+
+#include "fa_common.cuh"
+
+namespace fa {
+
+// Rescale O and l only when the running row max grew by more than this (log2 units);
+// until then P may reach 2^8, far inside fp32 / bf16 / fp16 range.
+constexpr float kRescaleTau = 8.0f;
+
+struct FwdParams {
+    void* o;
+    float* lse;
+    int B, Sq, Sk, Hq, Hkv, group;
+    int num_m;        // query blocks per head
+    int num_tiles;    // B * Hq * num_m
+    int chunk_heads;  // heads per L2 group in the unit order
+    int causal;
+    int inject;       // test hook: withhold the first K copy
+    float sl2;        // scale * log2(e)
+};
+
+// wait-site codes reported through the device status word
+enum : uint32_t {
+    W_FWD_Q_FULL = 0x101, W_FWD_Q_EMPTY, W_FWD_RING_FULL, W_FWD_RING_EMPTY, W_FWD_S_FULL,
+    W_FWD_P_FULL, W_FWD_O_DONE, W_FWD_O_FINAL, W_FWD_DRAIN
+};
+
+template <int D, bool BF16>
+struct FwdCfg {
+    static_assert(D == 128 || D == 256, "head_dim");
+    static constexpr int NQ = D == 128 ? 2 : 1;  // 128-row Q tiles per work unit
+    static constexpr int NS = D == 128 ? 1 : 2;  // S buffers per Q tile
+    static constexpr int KCH = D / 128;          // 32-KB chunks per K (or V) tile
+    static constexpr int NSTAGE = 5;             // ring depth, in chunks
+    static constexpr int BM = 128;               // query rows per Q tile
+    static constexpr int BN = 128;               // keys per KV tile
+    static constexpr int UNIT_ROWS = NQ * BM;
+    static constexpr uint32_t CHUNK = 32768;
+    static constexpr uint32_t QTILE = BM * D * 2;
+    static constexpr uint32_t Q_BYTES = NQ * QTILE;
+    static constexpr int THREADS = (NQ + 1) * 128;
+    static constexpr int CTRL_WARP = NQ * 4;  // MMA warp; the TMA warp follows it
+
+    // shared memory map (offsets from a 1024-aligned base)
+    static constexpr uint32_t OFF_Q = 0;
+    static constexpr uint32_t OFF_RING = Q_BYTES;
+    static constexpr uint32_t OFF_BAR = OFF_RING + NSTAGE * CHUNK;
+    // barrier indices
+    static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1;
+    static constexpr int B_FULL = 2;
+    static constexpr int B_EMPTY = B_FULL + NSTAGE;
+    static constexpr int B_S_FULL = B_EMPTY + NSTAGE;
+    static constexpr int B_P_FULL = B_S_FULL + NQ * NS;
+    static constexpr int B_O_DONE = B_P_FULL + NQ * NS;
+    static constexpr int B_O_FINAL = B_O_DONE + NQ;
+    static constexpr int B_DRAIN = B_O_FINAL + NQ;
+    static constexpr int NBAR = B_DRAIN + 1;
+    static constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
+    static constexpr uint32_t SMEM_BYTES = OFF_CTL + sizeof(CtaCtl) + 1024;
+
+    // TMEM columns
+    __device__ static constexpr uint32_t col_S(int q, int sb) { return NQ == 2 ? q * 128 : sb * 128; }
+    __device__ static constexpr uint32_t col_O(int q) { return 256 + q * 128; }
+
+    static constexpr uint32_t IDESC_S = idesc_f16(BF16, 128, 128, false, false);
+    static constexpr uint32_t IDESC_PV = idesc_f16(BF16, 128, 128, false, true);
+};
+
+template <int UNIT_ROWS>
+__device__ __forceinline__ void fwd_decode(const FwdParams& p, int t, int& b, int& h, int& m0)
+{
+    const int BH = p.B * p.Hq;
+    const int per_chunk = p.chunk_heads * p.num_m;
+    const int c = t / per_chunk;
+    const int r = t - c * per_chunk;
+    const int first = c * p.chunk_heads;
+    const int csize = min(p.chunk_heads, BH - first);
+    const int mi = r / csize;
+    const int bh = first + (r - mi * csize);
+    const int mblk = p.causal ? (p.num_m - 1 - mi) : mi;
+    b = bh / p.Hq;
+    h = bh - b * p.Hq;
+    m0 = mblk * UNIT_ROWS;
+}
+
+// Number of KV tiles a unit starting at query row m0 must visit.
+template <int UNIT_ROWS>
+__device__ __forceinline__ int fwd_kv_tiles(const FwdParams& p, int m0)
+{
+    const int nk = (p.Sk + 127) / 128;
+    if (!p.causal) return nk;
+    const int last_row = min(m0 + UNIT_ROWS, p.Sq) - 1;
+    const long long maxcol = static_cast<long long>(last_row) + p.Sk - p.Sq;
+    if (maxcol < 0) return 0;
+    return min(nk, static_cast<int>(maxcol / 128) + 1);
+}
+
+// ---------------------------------------------------------------------------------
+// Softmax / epilogue warpgroup (one per Q tile).
+// ---------------------------------------------------------------------------------
+template <int D, bool BF16>
+__device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int q,
+                            int wq)
+{
+    using C = FwdCfg<D, BF16>;
+    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    const int lane = threadIdx.x & 31;
+    const int r_in_tile = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tO = tmem + lane_off + C::col_O(q);
+    auto bar = [&](int i) { return bars + 8u * i; };
+    uint32_t s_it = 0, pv_it = 0, tile_it = 0;
+
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+        int b, h, m0;
+        fwd_decode<C::UNIT_ROWS>(p, t, b, h, m0);
+        const int n = fwd_kv_tiles<C::UNIT_ROWS>(p, m0);
+        const int q0 = m0 + q * C::BM;  // first query row of this Q tile
+        const int row = q0 + r_in_tile;
+        const bool row_ok = row < p.Sq;
+        T* orow = reinterpret_cast<T*>(p.o) + ((static_cast<size_t>(b) * p.Sq + row) * p.Hq + h) * D;
+        float* lrow = p.lse + (static_cast<size_t>(b) * p.Hq + h) * p.Sq + row;
+        if (n == 0) {  // causal with Sq > Sk: no key is visible to any row of the unit
+            if (row_ok) {
+                uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
+                *lrow = -INFINITY;
+            }
+            continue;
+        }
+        // columns >= lim are masked for this row; the tile-level test uses the first
+        // row of the Q tile, which has the smallest limit
+        const int lim = p.causal ? min(p.Sk, row + p.Sk - p.Sq + 1) : p.Sk;
+        const int lim0 = p.causal ? min(p.Sk, q0 + p.Sk - p.Sq + 1) : p.Sk;
+
+        float m_ref = -INFINITY;  // running reference max (log2 units)
+        float l = 0.0f;           // running row sum against m_ref
+        for (int j = 0; j < n; ++j) {
+            const int sb = s_it % C::NS;
+            if (!warp_wait(bar(C::B_S_FULL + q * C::NS + sb), (s_it / C::NS) & 1u, ctl, W_FWD_S_FULL))
+                return;
+            tc_fence_after();
+            const uint32_t tS = tmem + lane_off + C::col_S(q, sb);
+            uint32_t sr[128];
+            tmem_ld128_wait(tS, sr);
+            const bool masked = (j + 1) * C::BN > lim0;
+            if (masked) {
+                const int cut = lim - j * C::BN;
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c >= cut) sr[c] = __float_as_uint(-INFINITY);
+            }
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sr[i]);
+#pragma unroll
+            for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
+            const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float m_tile = rmax * p.sl2;  // scale > 0, so max commutes with it
+            const float m_new = fmaxf(m_ref, m_tile);
+            const bool resc = (m_ref != -INFINITY) && (m_new - m_ref > kRescaleTau);
+            if (m_ref == -INFINITY) m_ref = m_new;
+            if (__any_sync(0xffffffffu, resc)) {
+                // O must hold every earlier P V product before it is scaled: with one S
+                // buffer that is implied by S_full (the MMA issued S after the previous
+                // P V); with two, wait for the previous P V explicitly.
+                if (C::NS == 2) {
+                    if (!warp_wait(bar(C::B_O_DONE + q), (pv_it - 1u) & 1u, ctl, W_FWD_O_DONE)) return;
+                    tc_fence_after();
+                }
+                const float alpha = resc ? ex2_sfu(m_ref - m_new) : 1.0f;
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32_wait(tO + cc * 32, r);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+                    tmem_st32(tO + cc * 32, r);
+                }
+                tmem_wait_st();
+                if (resc) {
+                    l *= alpha;
+                    m_ref = m_new;
+                }
+            }
+            const float negm = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+            float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 32; k += 2) {
+                    const float x0 = fmaf(__uint_as_float(sr[cc * 32 + k]), p.sl2, negm);
+                    const float x1 = fmaf(__uint_as_float(sr[cc * 32 + k + 1]), p.sl2, negm);
+                    float e0, e1;
+                    // 1 of every 4 exponentials on the FMA pipe (unmasked tiles only:
+                    // the SFU maps -inf to exactly 0)
+                    if (!masked && (k & 2)) {
+                        e0 = exp2_fma(x0);
+                        e1 = ex2_sfu(x1);
+                    } else {
+                        e0 = ex2_sfu(x0);
+                        e1 = ex2_sfu(x1);
+                    }
+                    sum[(k >> 1) & 3] += e0 + e1;
+                    pk[k >> 1] = pack2<BF16>(e0, e1);
+                }
+                tmem_st16(tS + cc * 16, pk);
+            }
+            l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q * C::NS + sb));
+            ++s_it;
+            ++pv_it;
+        }
+        // epilogue: wait for the unit's last P V, normalise, store O and LSE
+        if (!warp_wait(bar(C::B_O_FINAL + q), tile_it & 1u, ctl, W_FWD_O_FINAL)) return;
+        ++tile_it;
+        tc_fence_after();
+        const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld32_wait(tO + cc * 32, r);
+            uint32_t pk[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                pk[k] = pack2<BF16>(__uint_as_float(r[2 * k]) * inv, __uint_as_float(r[2 * k + 1]) * inv);
+            if (row_ok) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+                dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+            }
+        }
+        if (row_ok) *lrow = (l > 0.0f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        tc_fence_before();
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// MMA issuer (one thread).
+// ---------------------------------------------------------------------------------
+template <int D, bool BF16>
+struct FwdMma {
+    using C = FwdCfg<D, BF16>;
+    uint32_t tmem, sQ, sRing, bars;
+    CtaCtl* ctl;
+    uint32_t seq = 0;  // ring chunk sequence number
+
+    __device__ uint32_t bar(int i) const { return bars + 8u * i; }
+    __device__ uint32_t slot(uint32_t s) const { return sRing + (s % C::NSTAGE) * C::CHUNK; }
+    __device__ bool wait_full(uint32_t s)
+    {
+        return wait_bar(bar(C::B_FULL + s % C::NSTAGE), (s / C::NSTAGE) & 1u, ctl, W_FWD_RING_FULL);
+    }
+    __device__ void release(uint32_t s) { mma_commit(bar(C::B_EMPTY + s % C::NSTAGE)); }
+
+    // S(q, sb) = Q_q K^T, K tile in ring chunks sK .. sK + KCH - 1
+    __device__ void issue_S(int q, int sb, uint32_t sK)
+    {
+        const uint32_t d = tmem + C::col_S(q, sb);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t a = sQ + q * C::QTILE + (kk >> 2) * 16384u + (kk & 3) * 32u;
+            const uint32_t bk = slot(sK + (kk >> 3)) + ((kk & 7) >> 2) * 16384u + (kk & 3) * 32u;
+            mma_ss(d, sdesc_sw128(a, 16, 1024), sdesc_sw128(bk, 16, 1024), C::IDESC_S, kk > 0);
+        }
+    }
+    // O_q (+)= P(q, sb) V, V tile in ring chunks sV .. sV + KCH - 1 (chunk c = O columns
+    // c*128 .. c*128+127)
+    __device__ void issue_PV(int q, int sb, uint32_t sV, bool acc)
+    {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t a = tmem + C::col_S(q, sb) + kk * 8;
+#pragma unroll
+            for (int c = 0; c < C::KCH; ++c) {
+                const uint32_t bv = slot(sV + c) + kk * 2048u;
+                mma_ts(tmem + C::col_O(q) + c * 128, a, sdesc_sw128(bv, 16384, 1024), C::IDESC_PV,
+                       (acc || kk > 0) ? 1u : 0u);
+            }
+        }
+    }
+    __device__ bool wait_chunks(uint32_t s0)
+    {
+        for (int c = 0; c < C::KCH; ++c)
+            if (!wait_full(s0 + c)) return false;
+        tc_fence_after();
+        return true;
+    }
+    __device__ void release_chunks(uint32_t s0)
+    {
+        for (int c = 0; c < C::KCH; ++c) release(s0 + c);
+    }
+
+    __device__ void run(const FwdParams& p)
+    {
+        uint32_t s_it[C::NQ] = {}, p_it[C::NQ] = {};
+        uint32_t q_it = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+            int b, h, m0;
+            fwd_decode<C::UNIT_ROWS>(p, t, b, h, m0);
+            const int n = fwd_kv_tiles<C::UNIT_ROWS>(p, m0);
+            if (n == 0) continue;
+            if (!wait_bar(bar(C::B_Q_FULL), q_it & 1u, ctl, W_FWD_Q_FULL)) return;
+            ++q_it;
+            tc_fence_after();
+            if constexpr (C::NQ == 2) {
+                // order per KV tile j: PV0(j-1), S0(j), PV1(j-1), S1(j)
+                uint32_t sK = seq;
+                seq += 1;
+                if (!wait_chunks(sK)) return;
+                for (int q = 0; q < 2; ++q) {
+                    issue_S(q, 0, sK);
+                    mma_commit(bar(C::B_S_FULL + q));
+                    ++s_it[q];
+                }
+                release(sK);
+                if (n == 1) mma_commit(bar(C::B_Q_EMPTY));
+                for (int j = 1; j < n; ++j) {
+                    const uint32_t sV = seq;
+                    seq += 1;
+                    if (!wait_chunks(sV)) return;
+                    if (!wait_bar(bar(C::B_P_FULL + 0), p_it[0] & 1u, ctl, W_FWD_P_FULL)) return;
+                    tc_fence_after();
+                    issue_PV(0, 0, sV, j > 1);
+                    ++p_it[0];
+                    sK = seq;
+                    seq += 1;
+                    if (!wait_chunks(sK)) return;
+                    issue_S(0, 0, sK);
+                    mma_commit(bar(C::B_S_FULL + 0));
+                    ++s_it[0];
+                    if (!wait_bar(bar(C::B_P_FULL + 1), p_it[1] & 1u, ctl, W_FWD_P_FULL)) return;
+                    tc_fence_after();
+                    issue_PV(1, 0, sV, j > 1);
+                    ++p_it[1];
+                    release(sV);
+                    issue_S(1, 0, sK);
+                    mma_commit(bar(C::B_S_FULL + 1));
+                    ++s_it[1];
+                    release(sK);
+                    if (j == n - 1) mma_commit(bar(C::B_Q_EMPTY));
+                }
+                const uint32_t sV = seq;
+                seq += 1;
+                if (!wait_chunks(sV)) return;
+                for (int q = 0; q < 2; ++q) {
+                    if (!wait_bar(bar(C::B_P_FULL + q), p_it[q] & 1u, ctl, W_FWD_P_FULL)) return;
+                    tc_fence_after();
+                    issue_PV(q, 0, sV, n > 1);
+                    ++p_it[q];
+                    mma_commit(bar(C::B_O_FINAL + q));
+                }
+                release(sV);
+            } else {
+                // one Q tile, two S buffers; order: S(0), S(1), then per j: PV(j), S(j+2)
+                for (int j = 0; j < 2 && j < n; ++j) {
+                    const uint32_t sK = seq;
+                    seq += C::KCH;
+                    if (!wait_chunks(sK)) return;
+                    const int sb = s_it[0] & 1;
+                    issue_S(0, sb, sK);
+                    mma_commit(bar(C::B_S_FULL + sb));
+                    ++s_it[0];
+                    release_chunks(sK);
+                }
+                if (n <= 2) mma_commit(bar(C::B_Q_EMPTY));
+                for (int j = 0; j < n; ++j) {
+                    const uint32_t sV = seq;
+                    seq += C::KCH;
+                    if (!wait_chunks(sV)) return;
+                    const int sbp = p_it[0] & 1;
+                    if (!wait_bar(bar(C::B_P_FULL + sbp), (p_it[0] >> 1) & 1u, ctl, W_FWD_P_FULL)) return;
+                    tc_fence_after();
+                    issue_PV(0, sbp, sV, j > 0);
+                    mma_commit(bar(C::B_O_DONE));
+                    ++p_it[0];
+                    release_chunks(sV);
+                    if (j + 2 < n) {
+                        const uint32_t sK = seq;
+                        seq += C::KCH;
+                        if (!wait_chunks(sK)) return;
+                        const int sb = s_it[0] & 1;
+                        issue_S(0, sb, sK);
+                        mma_commit(bar(C::B_S_FULL + sb));
+                        ++s_it[0];
+                        release_chunks(sK);
+                        if (j + 2 == n - 1) mma_commit(bar(C::B_Q_EMPTY));
+                    }
+                }
+                mma_commit(bar(C::B_O_FINAL));
+            }
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------------
+// TMA producer (one thread).  The chunk order must equal the MMA issuer's.
+// ---------------------------------------------------------------------------------
+template <int D, bool BF16>
+struct FwdLoad {
+    using C = FwdCfg<D, BF16>;
+    const CUtensorMap *tmQ, *tmK, *tmV;
+    uint32_t sQ, sRing, bars;
+    CtaCtl* ctl;
+    uint32_t seq = 0;
+    int filled[C::NSTAGE];  // ring round of the last fill per slot, -1 if none
+    int q_round = -1;
+    int inject = 0;
+
+    __device__ uint32_t bar(int i) const { return bars + 8u * i; }
+
+    __device__ bool load_chunk(const CUtensorMap* tm, int row0, int col0, int hkv, int b)
+    {
+        const uint32_t s = seq++;
+        const int slot = s % C::NSTAGE;
+        const uint32_t round = s / C::NSTAGE;
+        if (!wait_bar(bar(C::B_EMPTY + slot), (round & 1u) ^ 1u, ctl, W_FWD_RING_EMPTY)) return false;
+        if (inject) {  // test hook: never fill this chunk; its consumer times out
+            inject = 0;
+            return true;
+        }
+        const uint32_t dst = sRing + slot * C::CHUNK;
+        mbar_arrive_expect_tx(bar(C::B_FULL + slot), C::CHUNK);
+        tma_load_4d(dst, tm, bar(C::B_FULL + slot), col0, hkv, row0, b);
+        tma_load_4d(dst + 16384u, tm, bar(C::B_FULL + slot), col0 + 64, hkv, row0, b);
+        filled[slot] = static_cast<int>(round);
+        return true;
+    }
+    __device__ bool load_kv(const CUtensorMap* tm, int j, int hkv, int b)
+    {
+        for (int c = 0; c < C::KCH; ++c)
+            if (!load_chunk(tm, j * C::BN, c * 128, hkv, b)) return false;
+        return true;
+    }
+
+    __device__ void run(const FwdParams& p)
+    {
+        for (int i = 0; i < C::NSTAGE; ++i) filled[i] = -1;
+        inject = p.inject;
+        uint32_t q_it = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+            int b, h, m0;
+            fwd_decode<C::UNIT_ROWS>(p, t, b, h, m0);
+            const int n = fwd_kv_tiles<C::UNIT_ROWS>(p, m0);
+            if (n == 0) continue;
+            const int hkv = h / p.group;
+            if (!wait_bar(bar(C::B_Q_EMPTY), (q_it & 1u) ^ 1u, ctl, W_FWD_Q_EMPTY)) return;
+            mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_BYTES);
+            for (int q = 0; q < C::NQ; ++q)
+                for (int blk = 0; blk < D / 64; ++blk)
+                    tma_load_4d(sQ + q * C::QTILE + blk * 16384u, tmQ, bar(C::B_Q_FULL), blk * 64, h,
+                                m0 + q * C::BM, b);
+            q_round = static_cast<int>(q_it);
+            ++q_it;
+            if constexpr (C::NQ == 2) {
+                for (int j = 0; j < n; ++j) {
+                    if (!load_kv(tmK, j, hkv, b)) return;
+                    if (!load_kv(tmV, j, hkv, b)) return;
+                }
+            } else {
+                for (int j = 0; j < 2 && j < n; ++j)
+                    if (!load_kv(tmK, j, hkv, b)) return;
+                for (int j = 0; j < n; ++j) {
+                    if (!load_kv(tmV, j, hkv, b)) return;
+                    if (j + 2 < n && !load_kv(tmK, j + 2, hkv, b)) return;
+                }
+            }
+        }
+    }
+
+    // Before the CTA exits, wait for every copy this thread started (normally all
+    // were consumed already and these return at once).
+    __device__ void drain()
+    {
+        for (int i = 0; i < C::NSTAGE; ++i)
+            if (filled[i] >= 0) drain_wait(bar(C::B_FULL + i), static_cast<uint32_t>(filled[i]) & 1u, W_FWD_DRAIN);
+        if (q_round >= 0) drain_wait(bar(C::B_Q_FULL), static_cast<uint32_t>(q_round) & 1u, W_FWD_DRAIN);
+    }
+};
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p)
+{
+    using C = FwdCfg<D, BF16>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* base_ptr = smem_raw + (base - raw);
+    const uint32_t sQ = base + C::OFF_Q;
+    const uint32_t sRing = base + C::OFF_RING;
+    const uint32_t bars = base + C::OFF_BAR;
+    CtaCtl* ctl = reinterpret_cast<CtaCtl*>(base_ptr + C::OFF_CTL);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        auto bar = [&](int i) { return bars + 8u * i; };
+        mbar_init(bar(C::B_Q_FULL), 1);
+        mbar_init(bar(C::B_Q_EMPTY), 1);
+        for (int i = 0; i < C::NSTAGE; ++i) {
+            mbar_init(bar(C::B_FULL + i), 1);
+            mbar_init(bar(C::B_EMPTY + i), 1);
+        }
+        for (int i = 0; i < C::NQ * C::NS; ++i) {
+            mbar_init(bar(C::B_S_FULL + i), 1);
+            mbar_init(bar(C::B_P_FULL + i), 4);  // one arrive per softmax warp
+        }
+        for (int q = 0; q < C::NQ; ++q) {
+            mbar_init(bar(C::B_O_DONE + q), 1);
+            mbar_init(bar(C::B_O_FINAL + q), 1);
+        }
+        mbar_init(bar(C::B_DRAIN), 1);
+        ctl->abort = 0u;
+        fence_mbar_init();
+    }
+    if (warp == C::CTRL_WARP) {
+        tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+        tmem_relinquish();
+    }
+    if (warp == C::CTRL_WARP + 1 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp < C::NQ * 4) {
+        fwd_softmax<D, BF16>(p, tmem, bars, ctl, warp >> 2, warp & 3);
+    } else if (warp == C::CTRL_WARP) {
+        if (lane == 0) {
+            FwdMma<D, BF16> mma{tmem, sQ, sRing, bars, ctl};
+            mma.run(p);
+            // all MMAs issued by this thread must finish before TMEM is released
+            mma_commit(bars + 8u * C::B_DRAIN);
+            drain_wait(bars + 8u * C::B_DRAIN, 0u, W_FWD_DRAIN);
+        }
+        __syncwarp();
+    } else if (warp == C::CTRL_WARP + 1) {
+        if (lane == 0) {
+            FwdLoad<D, BF16> ld{&tmQ, &tmK, &tmV, sQ, sRing, bars, ctl};
+            ld.run(p);
+            ld.drain();
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == C::CTRL_WARP) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace fa

@@ -1,0 +1,112 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library, libfa.so.
+ *
+ * Operation: exact scaled-dot-product attention and its backward,
+ *     O   = softmax(scale * Q K^T [+ causal mask]) V
+ *     LSE = log-sum-exp of the scaled, masked scores of each query row
+ * computed tile by tile with an online softmax so that the score matrix never
+ * reaches device memory ("FlashAttention 4: Snellere, Geheugenefficiente Aandacht
+ * voor LLM's", introduction and sections "Wat is nieuw in FlashAttention 4",
+ * "Software-exponentials via CUDA-kernen", "Slimmere Online
+ * Softmax-herwaardering"; the backward is listed as merged for SM100 in
+ * "[RFC] FA4 -- head_dim=256 & head_dim=512", Phase 1 table).
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense, contiguous, row-major [batch, seq, heads, head_dim] in
+ *     device memory ("h3-blackwell-runtime/FLASH4.md", section "API": the
+ *     kernel is called in that native layout with FP16/BF16 inputs).
+ *     Q, O, dO, dQ have Hq heads and Sq rows; K, V, dK, dV have Hkv heads and
+ *     Sk rows.  LSE is float32 [batch, Hq, Sq] holding the natural-log
+ *     log-sum-exp of scale * q.k over the visible keys (-inf for a row that sees
+ *     no key).
+ *   - Grouped-query attention: Hq must be a multiple of Hkv, and query head h
+ *     reads key/value head h / (Hq / Hkv).
+ *   - causal != 0 applies a lower-triangular mask aligned to the bottom-right
+ *     corner: key j is visible to query i iff j <= i + (Sk - Sq).
+ *   - head_dim d must be 128 or 256; dtype must be FA_BF16 or FA_FP16 and is
+ *     the same for every 16-bit tensor of a call.  Every pointer must be
+ *     16-byte aligned.
+ *   - Ownership: the caller owns every buffer.  The library allocates no device
+ *     memory per call; scratch for the backward is the caller's workspace.
+ *     Work is enqueued on `stream` and runs asynchronously; nothing synchronises.
+ *   - Errors: an invalid argument returns a status and launches nothing.  There
+ *     is no fallback path of any kind ("h3-blackwell-runtime/FLASH4.md": any
+ *     violation raises an error instead of changing kernels).
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,    /* a size, pointer, alignment or scale is invalid          */
+    FA_ERR_UNSUPPORTED = 2,    /* head_dim, dtype or GPU architecture not supported       */
+    FA_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed                       */
+    FA_ERR_DEVICE_TIMEOUT = 4  /* a kernel gave up on a bounded wait (see status query)   */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/* Opaque CUDA stream handle (cudaStream_t); 0 is the legacy default stream. */
+typedef void* fa_stream;
+
+/*
+ * Forward.  q [B,Sq,Hq,d], k/v [B,Sk,Hkv,d] -> o [B,Sq,Hq,d] (same dtype),
+ * lse [B,Hq,Sq] float32.  scale must be finite and > 0 (1/sqrt(d) is the usual
+ * choice).  Sizes: B, Sq, Sk, Hq, Hkv >= 1.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Sq, int Sk, int Hq, int Hkv, int d, int causal, float scale,
+                 fa_dtype dt, fa_stream stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for these sizes: the row terms
+ * D = rowsum(dO * O), the log2-domain LSE copy and the float32 dQ accumulator.
+ */
+size_t fa_bwd_workspace_size(int B, int Sq, int Hq, int d);
+
+/*
+ * Backward.  Given the forward's inputs q, k, v, its outputs o and lse, and the
+ * output gradient dO (same layout as o), writes dq [B,Sq,Hq,d], dk/dv
+ * [B,Sk,Hkv,d] in the input dtype.  `workspace` is caller-owned device memory of
+ * at least fa_bwd_workspace_size(B, Sq, Hq, d) bytes, 256-byte aligned; its
+ * contents on entry do not matter and are overwritten.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv,
+                 int B, int Sq, int Sk, int Hq, int Hkv, int d, int causal, float scale,
+                 fa_dtype dt, void* workspace, size_t workspace_bytes, fa_stream stream);
+
+/* Static, human-readable name of a status code. */
+const char* fa_status_string(fa_status s);
+
+/*
+ * Device-side status of the kernels run so far on this device: FA_OK, or
+ * FA_ERR_DEVICE_TIMEOUT if some kernel gave up on a bounded wait (each wait in
+ * the kernels gives up after about one second).  Synchronises `stream` to read
+ * it.  `detail` (may be NULL) receives a code naming the wait that gave up.
+ */
+fa_status fa_last_device_status(fa_stream stream, uint32_t* detail);
+
+/* Resets the device-side status to FA_OK (enqueued on `stream`). */
+fa_status fa_clear_device_status(fa_stream stream);
+
+/*
+ * Test hook: when `mode` is 1, the next forward launch withholds its first K
+ * tile copy so that the consumer's bounded wait runs out and the kernel reports
+ * FA_ERR_DEVICE_TIMEOUT instead of hanging.  The hook disarms itself after one
+ * launch.  0 disarms it.
+ */
+fa_status fa_debug_inject(int mode);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

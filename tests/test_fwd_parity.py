@@ -1,0 +1,96 @@
+"""GPU parity of fa_fwd against the fp64 oracle (element by element).
+
+Tolerances: O max abs error <= 1e-2 and mean abs error <= 1e-3, LSE abs error
+<= 1e-3, on 16-bit inputs drawn N(0, 1) (0.5 N(0, 1) for the video shapes).
+Rows that see no key (causal with Sq > Sk) must give O = 0 and LSE = -inf.
+"""
+import math
+
+import pytest
+import torch
+
+from exact_attention_blackwell_fa_b200.inputs import Shape, make_inputs, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+O_MAX, O_MEAN, LSE_MAX = 1e-2, 1e-3, 1e-3
+
+
+def run_fwd(shape, causal, dtype=torch.bfloat16, amp=1.0, seed=0, scale=None):
+    import exact_attention_blackwell_fa_b200 as fa
+
+    q, k, v = make_inputs(shape, seed=seed, dtype=dtype, amp=amp)
+    o, lse = fa.fa_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    return (q, k, v), o.cpu(), lse.cpu()
+
+
+def check_full(oracle_mod, shape, causal, dtype=torch.bfloat16, amp=1.0, scale=None):
+    (q, k, v), o, lse = run_fwd(shape, causal, dtype, amp, scale=scale)
+    o_ref, lse_ref = oracle_mod.fwd(q, k, v, causal=causal, scale=scale)
+    err = (o.double() - o_ref).abs()
+    assert torch.isfinite(o.double()).all()
+    assert err.max().item() <= O_MAX, f"O max abs err {err.max().item()}"
+    assert err.mean().item() <= O_MEAN, f"O mean abs err {err.mean().item()}"
+    fin = torch.isfinite(lse_ref)
+    assert torch.equal(torch.isfinite(lse), fin), "LSE -inf pattern differs"
+    if fin.any():
+        lerr = (lse.double()[fin] - lse_ref[fin]).abs().max().item()
+        assert lerr <= LSE_MAX, f"LSE abs err {lerr}"
+    assert torch.all(torch.isneginf(lse[~fin]))
+    return err.max().item()
+
+
+SMALL = [
+    # B, Sq, Sk, Hq, Hkv, d
+    (1, 256, 256, 2, 2, 128),      # the small forward configuration
+    (2, 384, 384, 2, 2, 128),
+    (1, 300, 200, 4, 2, 128),      # ragged tails, Sq != Sk, GQA
+    (1, 200, 333, 4, 1, 128),
+    (1, 256, 256, 2, 2, 256),
+    (2, 300, 520, 2, 1, 256),
+    (1, 1, 1, 1, 1, 128),
+    (1, 1, 1, 1, 1, 256),
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SMALL)
+def test_fwd_small_bf16(oracle_mod, shape, causal):
+    check_full(oracle_mod, Shape(*shape), causal)
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_fwd_fp16(oracle_mod, d):
+    check_full(oracle_mod, Shape(1, 320, 320, 2, 2, d), True, dtype=torch.float16)
+    check_full(oracle_mod, Shape(1, 320, 320, 2, 2, d), False, dtype=torch.float16)
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_fwd_causal_rows_without_keys(oracle_mod, d):
+    """Causal with Sq much larger than Sk: whole units see no key at all."""
+    check_full(oracle_mod, Shape(1, 700, 100, 2, 1, d), True)
+
+
+def test_fwd_video_small(oracle_mod):
+    """[1, 257, 8, 128] video-diffusion shape, inputs 0.5 N(0, 1)."""
+    check_full(oracle_mod, Shape(1, 257, 257, 8, 8, 128), False, amp=0.5)
+
+
+def test_fwd_custom_scale(oracle_mod):
+    check_full(oracle_mod, Shape(1, 256, 384, 2, 2, 128), False, scale=0.3)
+    check_full(oracle_mod, Shape(1, 256, 384, 2, 2, 256), True, scale=0.05)
+
+
+def test_fwd_many_units_persistent(oracle_mod):
+    """More work units than SMs so each persistent CTA walks several units."""
+    shape = Shape(2, 1024, 1024, 96, 24, 128)          # 2*96*4 = 768 units
+    (q, k, v), o, lse = run_fwd(shape, True)
+    rows = sample_rows(2, 96, 1024, 6, seed=5)
+    o_ref, lse_ref = oracle_mod.fwd(q, k, v, causal=True, rows=rows)
+    got = o[rows[:, 0], rows[:, 2], rows[:, 1]].double()
+    err = (got - o_ref).abs()
+    assert err.max().item() <= O_MAX
+    assert err.mean().item() <= O_MEAN
+    lerr = (lse[rows[:, 0], rows[:, 1], rows[:, 2]].double() - lse_ref).abs().max().item()
+    assert lerr <= LSE_MAX
