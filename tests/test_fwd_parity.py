@@ -25,12 +25,22 @@ def run_fwd(shape, causal, dtype=torch.bfloat16, amp=1.0, seed=0, scale=None):
     return (q, k, v), o.cpu(), lse.cpu()
 
 
+def p_rounding_bound(v, dtype):
+    """Largest O error the 16-bit rounding of P alone can cause: P is rounded to the
+    input dtype before the P V product (unit roundoff u = 2^-8 for bf16, 2^-11 for
+    fp16), so |dO_i| <= u * sum_j P_ij |v_j| <= u * max |v|.  Used where the scale
+    differs from 1/sqrt(d), which sharpens the softmax beyond the N(0, 1) tolerance."""
+    u = 2.0 ** -8 if dtype == torch.bfloat16 else 2.0 ** -11
+    return u * v.double().abs().max().item() + 1e-3
+
+
 def check_full(oracle_mod, shape, causal, dtype=torch.bfloat16, amp=1.0, scale=None):
     (q, k, v), o, lse = run_fwd(shape, causal, dtype, amp, scale=scale)
     o_ref, lse_ref = oracle_mod.fwd(q, k, v, causal=causal, scale=scale)
     err = (o.double() - o_ref).abs()
     assert torch.isfinite(o.double()).all()
-    assert err.max().item() <= O_MAX, f"O max abs err {err.max().item()}"
+    o_max = O_MAX if scale is None else max(O_MAX, p_rounding_bound(v, dtype))
+    assert err.max().item() <= o_max, f"O max abs err {err.max().item()}"
     assert err.mean().item() <= O_MEAN, f"O mean abs err {err.mean().item()}"
     fin = torch.isfinite(lse_ref)
     assert torch.equal(torch.isfinite(lse), fin), "LSE -inf pattern differs"
