@@ -125,6 +125,25 @@ int take_inject()
     return v;
 }
 
+template <bool BF16>
+fa_status launch_bwd_d128(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const fa::BwdParams& p, int sm_count,
+                          cudaStream_t stream)
+{
+    using C = fa::BwdCfg<BF16>;
+    const long long pre_rows = (long long)p.B * p.Hq * p.Sq_pad;
+    fa::fa_bwd_pre_kernel<128, BF16><<<(unsigned)((pre_rows + 7) / 8), 256, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    fa_status st = set_smem(fa::fa_bwd_dkdv_kernel<BF16>, C::SMEM_BYTES);
+    if (st != FA_OK) return st;
+    const int grid = p.num_units < sm_count ? p.num_units : sm_count;
+    fa::fa_bwd_dkdv_kernel<BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    const long long dq_rows = (long long)p.B * p.Sq * p.Hq;
+    fa::fa_bwd_dq_kernel<128, BF16><<<(unsigned)((dq_rows + 7) / 8), 256, 0, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 template <int D, bool BF16>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      fa::FwdParams p, int sm_count, cudaStream_t stream)
@@ -205,9 +224,49 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     DeviceInfo di;
     st = device_info(&di);
     if (st != FA_OK) return st;
-    return fa::launch_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Sq, Sk, Hq, Hkv, d, causal != 0,
-                          scale, dt == FA_BF16, workspace, di.sm_count,
-                          reinterpret_cast<cudaStream_t>(stream));
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    const bool bf16 = dt == FA_BF16;
+    CUtensorMap tq, tk, tv, tdo;
+    if (!make_tmap(&tq, q, B, Sq, Hq, d, bf16) || !make_tmap(&tk, k, B, Sk, Hkv, d, bf16) ||
+        !make_tmap(&tv, v, B, Sk, Hkv, d, bf16) || !make_tmap(&tdo, dout, B, Sq, Hq, d, bf16))
+        return FA_ERR_CUDA;
+    fa::BwdParams p{};
+    p.o = o;
+    p.dout = dout;
+    p.lse = lse;
+    const size_t sq_pad = fa::bwd_sq_pad(Sq);
+    const size_t rows = (size_t)B * Hq * sq_pad;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.Dv = reinterpret_cast<float*>(ws);
+    p.L2 = reinterpret_cast<float*>(ws + fa::bwd_round256(rows * 4));
+    p.dqacc = reinterpret_cast<float*>(ws + 2 * fa::bwd_round256(rows * 4));
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.B = B;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.group = Hq / Hkv;
+    p.Sq_pad = (int)sq_pad;
+    p.num_n = (Sk + 127) / 128;
+    p.num_m = (Sq + 127) / 128;
+    p.num_units = B * Hkv * p.num_n;
+    // KV heads whose Q and dO streams stay inside L2 together
+    {
+        const double qdo_bytes = 2.0 * Sq * d * 2.0 * p.group;
+        int c = (int)(48.0 * 1024 * 1024 / (qdo_bytes > 1.0 ? qdo_bytes : 1.0));
+        if (c < 1) c = 1;
+        if (c > B * Hkv) c = B * Hkv;
+        p.chunk_heads = c;
+    }
+    p.causal = causal ? 1 : 0;
+    p.scale = scale;
+    p.sl2 = scale * 1.4426950408889634f;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return bf16 ? launch_bwd_d128<true>(tq, tk, tv, tdo, p, di.sm_count, s)
+                : launch_bwd_d128<false>(tq, tk, tv, tdo, p, di.sm_count, s);
 }
 
 const char* fa_status_string(fa_status s)

@@ -1,5 +1,29 @@
-// fa_bwd.cuh -- exact attention backward for sm_100a (placeholder until the kernels land).
+// fa_bwd.cuh -- exact attention backward for sm_100a.
+//
+// Given Q, K, V, O, LSE and dO, computes dQ, dK, dV of O = softmax(scale Q K^T) V
+// (the backward is listed as merged for SM100 in "[RFC] FA4 -- head_dim=256 &
+// head_dim=512", Phase 1 table; the arithmetic is the chain rule of the forward):
+//
+//   P_ij  = exp(scale q_i.k_j - LSE_i)          (recomputed, never stored in HBM)
+//   dP_ij = dO_i . v_j,   D_i = dO_i . O_i,   dS_ij = P_ij (dP_ij - D_i)
+//   dV_j  = sum_i P_ij dO_i,  dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j
+//
+// Three kernels on one stream:
+//   1. preprocess: D_i = rowsum(dO * O), LSE in log2 units, zero the fp32 dQ
+//      accumulator (rows padded to a multiple of 128);
+//   2. dK/dV kernel, persistent, one work unit = one block of 128 key rows of one
+//      (batch, KV head); it loops over every query head of the KV group and every
+//      block of 128 query rows.  Per step, all in TMEM:
+//        S^T = K Q^T,  dP^T = V dO^T            (tcgen05, A and B K-major)
+//        compute warpgroup (thread = key row): P^T -> TMEM as 16-bit pairs,
+//                                               dS^T -> shared memory (swizzled)
+//        dV += P^T dO   (A from TMEM)           dK += dS^T Q   (A K-major)
+//        dQ_part = dS K (A = the same dS^T tile read MN-major) -> TMEM -> fp32
+//        vector reductions into the dQ accumulator by a second warpgroup;
+//   3. convert: dQ = scale * accumulator, in the input dtype and layout.
 #pragma once
+
+#include <type_traits>
 
 #include "fa_common.cuh"
 
@@ -7,18 +31,562 @@ namespace fa {
 
 inline size_t bwd_round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+inline size_t bwd_sq_pad(int Sq) { return (static_cast<size_t>(Sq) + 127) / 128 * 128; }
+
+// workspace = D [B*Hq*Sq_pad] fp32 | LSE*log2(e) [B*Hq*Sq_pad] fp32 | dQacc [.. x d] fp32
 inline size_t bwd_workspace_bytes(int B, int Sq, int Hq, int d)
 {
-    const size_t sq_pad = (static_cast<size_t>(Sq) + 127) / 128 * 128;
-    const size_t rows = static_cast<size_t>(B) * Hq * sq_pad;
+    const size_t rows = static_cast<size_t>(B) * Hq * bwd_sq_pad(Sq);
     return 2 * bwd_round256(rows * 4) + bwd_round256(rows * d * 4);
 }
 
-inline fa_status launch_bwd(const void*, const void*, const void*, const void*, const float*,
-                            const void*, void*, void*, void*, int, int, int, int, int, int, bool,
-                            float, bool, void*, int, cudaStream_t)
+struct BwdParams {
+    const void* o;
+    const void* dout;
+    const float* lse;
+    float* Dv;     // D_i, padded rows 0
+    float* L2;     // LSE_i * log2(e); +inf for padded rows and rows without keys
+    float* dqacc;  // [B, Hq, Sq_pad, d] fp32
+    void* dq;
+    void* dk;
+    void* dv;
+    int B, Sq, Sk, Hq, Hkv, group, Sq_pad;
+    int num_n;        // key blocks per KV head
+    int num_m;        // query blocks per query head
+    int num_units;    // B * Hkv * num_n
+    int chunk_heads;  // KV heads per L2 group in the unit order
+    int causal;
+    float scale, sl2;
+};
+
+enum : uint32_t {
+    W_BWD_KV_FULL = 0x201, W_BWD_KV_EMPTY, W_BWD_Q_FULL, W_BWD_Q_EMPTY, W_BWD_DO_FULL,
+    W_BWD_DO_EMPTY, W_BWD_S_FULL, W_BWD_DP_FULL, W_BWD_P_FULL, W_BWD_DS_FULL, W_BWD_DS_EMPTY,
+    W_BWD_DQ_FULL, W_BWD_DQ_EMPTY, W_BWD_DKV_FINAL, W_BWD_DRAIN
+};
+
+// ---------------------------------------------------------------------------------
+// 1. preprocess: one warp per padded query row (b, h, i)
+// ---------------------------------------------------------------------------------
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p)
 {
-    return FA_ERR_UNSUPPORTED;
+    const int lane = threadIdx.x & 31;
+    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const long long total = static_cast<long long>(p.B) * p.Hq * p.Sq_pad;
+    if (row >= total) return;
+    const int bh = static_cast<int>(row / p.Sq_pad);
+    const int i = static_cast<int>(row - static_cast<long long>(bh) * p.Sq_pad);
+    const int b = bh / p.Hq, h = bh - b * p.Hq;
+    float acc = 0.0f;
+    if (i < p.Sq) {
+        const size_t off = ((static_cast<size_t>(b) * p.Sq + i) * p.Hq + h) * D + lane * (D / 32);
+        constexpr int NW = D / 64;  // 32-bit words per lane (two 16-bit values each)
+        uint32_t ow[NW], dw[NW];
+        if constexpr (NW == 2) {
+            const uint2 a = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.o) + off);
+            const uint2 c = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.dout) + off);
+            ow[0] = a.x; ow[1] = a.y; dw[0] = c.x; dw[1] = c.y;
+        } else {
+            const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + off);
+            const uint4 c = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + off);
+            ow[0] = a.x; ow[1] = a.y; ow[2] = a.z; ow[3] = a.w;
+            dw[0] = c.x; dw[1] = c.y; dw[2] = c.z; dw[3] = c.w;
+        }
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float2 x = unpack2<BF16>(ow[w]);
+            const float2 y = unpack2<BF16>(dw[w]);
+            acc = fmaf(x.x, y.x, acc);
+            acc = fmaf(x.y, y.y, acc);
+        }
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (lane == 0) {
+        p.Dv[row] = acc;
+        float l2 = INFINITY;
+        if (i < p.Sq) {
+            const float lse = p.lse[static_cast<size_t>(bh) * p.Sq + i];
+            if (lse != -INFINITY) l2 = lse * 1.4426950408889634f;
+        }
+        p.L2[row] = l2;
+    }
+    float4* z = reinterpret_cast<float4*>(p.dqacc + static_cast<size_t>(row) * D);
+#pragma unroll
+    for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ---------------------------------------------------------------------------------
+// 3. convert: one warp per dQ row (b, i, h)
+// ---------------------------------------------------------------------------------
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p)
+{
+    const int lane = threadIdx.x & 31;
+    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const long long total = static_cast<long long>(p.B) * p.Sq * p.Hq;
+    if (row >= total) return;
+    const int h = static_cast<int>(row % p.Hq);
+    const long long bi = row / p.Hq;
+    const int i = static_cast<int>(bi % p.Sq);
+    const int b = static_cast<int>(bi / p.Sq);
+    const float* src = p.dqacc + ((static_cast<size_t>(b) * p.Hq + h) * p.Sq_pad + i) * D + lane * (D / 32);
+    uint16_t* dst = static_cast<uint16_t*>(p.dq) + static_cast<size_t>(row) * D + lane * (D / 32);
+    if constexpr (D == 128) {
+        const float4 a = *reinterpret_cast<const float4*>(src);
+        *reinterpret_cast<uint2*>(dst) =
+            make_uint2(pack2<BF16>(a.x * p.scale, a.y * p.scale), pack2<BF16>(a.z * p.scale, a.w * p.scale));
+    } else {
+        const float4 a = reinterpret_cast<const float4*>(src)[0];
+        const float4 c = reinterpret_cast<const float4*>(src)[1];
+        *reinterpret_cast<uint4*>(dst) =
+            make_uint4(pack2<BF16>(a.x * p.scale, a.y * p.scale), pack2<BF16>(a.z * p.scale, a.w * p.scale),
+                       pack2<BF16>(c.x * p.scale, c.y * p.scale), pack2<BF16>(c.z * p.scale, c.w * p.scale));
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// 2. dK / dV kernel (head_dim 128)
+// ---------------------------------------------------------------------------------
+template <bool BF16>
+struct BwdCfg {
+    static constexpr int D = 128;
+    static constexpr int THREADS = 384;
+    static constexpr int MMA_WARP = 8, LOAD_WARP = 9;
+    static constexpr uint32_t TILE = 32768;  // 128 rows x 128 columns x 2 bytes
+    static constexpr uint32_t OFF_K = 0, OFF_V = TILE, OFF_Q = 2 * TILE, OFF_DO = 4 * TILE,
+                              OFF_DS = 6 * TILE, OFF_BAR = 7 * TILE;
+    static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1, B_Q_FULL = 2, B_Q_EMPTY = 4, B_DO_FULL = 6,
+                         B_DO_EMPTY = 8, B_S_FULL = 10, B_DP_FULL = 11, B_P_FULL = 12, B_DS_FULL = 13,
+                         B_DS_EMPTY = 14, B_DQ_FULL = 15, B_DQ_EMPTY = 16, B_DKV_FINAL = 17,
+                         B_DRAIN = 18, NBAR = 19;
+    static constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
+    static constexpr uint32_t SMEM_BYTES = OFF_CTL + sizeof(CtaCtl) + 1024;
+    // TMEM columns
+    static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
+    static constexpr uint32_t IDESC_KK = idesc_f16(BF16, 128, 128, false, false);  // S^T, dP^T
+    static constexpr uint32_t IDESC_KM = idesc_f16(BF16, 128, 128, false, true);   // dV, dK
+    static constexpr uint32_t IDESC_MM = idesc_f16(BF16, 128, 128, true, true);    // dQ
+};
+
+struct BwdUnit {
+    int b, hkv, n, m_start, nm, T;
+};
+
+__device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int t)
+{
+    const int BH = p.B * p.Hkv;
+    const int per_chunk = p.chunk_heads * p.num_n;
+    const int c = t / per_chunk;
+    const int r = t - c * per_chunk;
+    const int first = c * p.chunk_heads;
+    const int csize = min(p.chunk_heads, BH - first);
+    const int nb = r / csize;  // causal: ascending n = most query blocks first
+    const int bh = first + (r - nb * csize);
+    BwdUnit u;
+    u.b = bh / p.Hkv;
+    u.hkv = bh - u.b * p.Hkv;
+    u.n = nb;
+    int ms = 0;
+    if (p.causal) {
+        const long long imin = static_cast<long long>(u.n) * 128 - (p.Sk - p.Sq);
+        ms = imin <= 0 ? 0 : static_cast<int>(imin / 128);
+        if (ms > p.num_m) ms = p.num_m;
+    }
+    u.m_start = ms;
+    u.nm = p.num_m - ms;
+    u.T = p.group * u.nm;
+    return u;
+}
+
+// query head and query block of step s of a unit
+__device__ __forceinline__ void bwd_step(const BwdParams& p, const BwdUnit& u, int s, int& h, int& m)
+{
+    const int hh = s / u.nm;
+    m = u.m_start + (s - hh * u.nm);
+    h = u.hkv * p.group + hh;
+}
+
+// ---- compute warpgroup: P^T and dS^T, then the dK / dV epilogue --------------------
+template <bool BF16>
+__device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uint32_t bars,
+                            CtaCtl* ctl, int wq)
+{
+    using C = BwdCfg<BF16>;
+    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    const int lane = threadIdx.x & 31;
+    const int t = wq * 32 + lane;  // key row within the block (= TMEM lane)
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    auto bar = [&](int i) { return bars + 8u * i; };
+    uint32_t it = 0, unit_it = 0;
+    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+        const BwdUnit u = bwd_decode(p, ui);
+        const int j = u.n * 128 + t;  // key row
+        for (int s = 0; s < u.T; ++s, ++it) {
+            int h, m;
+            bwd_step(p, u, s, h, m);
+            const size_t rbase = (static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + static_cast<size_t>(m) * 128;
+            const float4* L2v = reinterpret_cast<const float4*>(p.L2 + rbase);
+            const float4* Dvv = reinterpret_cast<const float4*>(p.Dv + rbase);
+            // key j is visible to query i iff j <= i + (Sk - Sq)
+            const bool masked = p.causal && (u.n * 128 + 127 > m * 128 + p.Sk - p.Sq);
+            const int jlim = j - (p.Sk - p.Sq) - m * 128;  // visible iff column c >= jlim
+            if (!warp_wait(bar(C::B_S_FULL), it & 1u, ctl, W_BWD_S_FULL)) return;
+            tc_fence_after();
+            float P[128];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t r[32];
+                tmem_ld32_wait(tmem + lane_off + C::T_S + cc * 32, r);
+                uint32_t pk[16];
+#pragma unroll
+                for (int k4 = 0; k4 < 8; ++k4) {
+                    const float4 l4 = L2v[cc * 8 + k4];
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = cc * 32 + k4 * 4 + e;
+                        const float x = fmaf(__uint_as_float(r[k4 * 4 + e]), p.sl2, -lv[e]);
+                        float pv = ((e & 1) && !masked) ? exp2_fma(x) : ex2_sfu(x);
+                        if (masked && c < jlim) pv = 0.0f;
+                        P[c] = pv;
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k) pk[k] = pack2<BF16>(P[cc * 32 + 2 * k], P[cc * 32 + 2 * k + 1]);
+                tmem_st16(tmem + lane_off + C::T_S + cc * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_P_FULL));
+
+            if (!warp_wait(bar(C::B_DP_FULL), it & 1u, ctl, W_BWD_DP_FULL)) return;
+            if (!warp_wait(bar(C::B_DS_EMPTY), (it & 1u) ^ 1u, ctl, W_BWD_DS_EMPTY)) return;
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t r[32];
+                tmem_ld32_wait(tmem + lane_off + C::T_DP + cc * 32, r);
+                uint32_t pk[16];
+#pragma unroll
+                for (int k4 = 0; k4 < 8; ++k4) {
+                    const float4 d4 = Dvv[cc * 8 + k4];
+                    const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float ds[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = cc * 32 + k4 * 4 + e;
+                        ds[e] = P[c] * (__uint_as_float(r[k4 * 4 + e]) - dv[e]);
+                    }
+                    pk[k4 * 2] = pack2<BF16>(ds[0], ds[1]);
+                    pk[k4 * 2 + 1] = pack2<BF16>(ds[2], ds[3]);
+                }
+                // columns cc*32 .. cc*32+31 = four 16-byte chunks of row t, 128-byte swizzle
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int col8 = cc * 4 + g;  // 8-column group 0..15
+                    const uint32_t addr = sDS + (col8 >> 3) * 16384u + t * 128u +
+                                          ((static_cast<uint32_t>(col8 & 7) ^ (t & 7)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                 "r"(pk[4 * g]), "r"(pk[4 * g + 1]), "r"(pk[4 * g + 2]), "r"(pk[4 * g + 3])
+                                 : "memory");
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_DS_FULL));
+        }
+        // epilogue: dV and dK rows of this key block
+        if (!warp_wait(bar(C::B_DKV_FINAL), unit_it & 1u, ctl, W_BWD_DKV_FINAL)) return;
+        ++unit_it;
+        tc_fence_after();
+        const bool row_ok = j < p.Sk;
+        const size_t off = ((static_cast<size_t>(u.b) * p.Sk + j) * p.Hkv + u.hkv) * C::D;
+        T* dvrow = static_cast<T*>(p.dv) + off;
+        T* dkrow = static_cast<T*>(p.dk) + off;
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+            const float mul = which == 0 ? 1.0f : p.scale;
+            T* dst = which == 0 ? dvrow : dkrow;
+            const uint32_t col = which == 0 ? C::T_DV : C::T_DK;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t r[32];
+                tmem_ld32_wait(tmem + lane_off + col + cc * 32, r);
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    pk[k] = pack2<BF16>(__uint_as_float(r[2 * k]) * mul, __uint_as_float(r[2 * k + 1]) * mul);
+                if (row_ok) {
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+                    d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    d4[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+                    d4[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+                }
+            }
+        }
+        tc_fence_before();
+    }
+}
+
+// ---- dQ warpgroup: TMEM -> registers -> fp32 vector reductions ----------------------
+template <bool BF16>
+__device__ void bwd_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int wq)
+{
+    using C = BwdCfg<BF16>;
+    const int lane = threadIdx.x & 31;
+    const int t = wq * 32 + lane;  // query row within the block
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    auto bar = [&](int i) { return bars + 8u * i; };
+    uint32_t it = 0;
+    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+        const BwdUnit u = bwd_decode(p, ui);
+        for (int s = 0; s < u.T; ++s, ++it) {
+            int h, m;
+            bwd_step(p, u, s, h, m);
+            if (!warp_wait(bar(C::B_DQ_FULL), it & 1u, ctl, W_BWD_DQ_FULL)) return;
+            tc_fence_after();
+            uint32_t r[128];
+            tmem_ld128_wait(tmem + lane_off + C::T_DP, r);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
+            float* dst = p.dqacc + ((static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + m * 128 + t) * C::D;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * c),
+                             "f"(__uint_as_float(r[4 * c])), "f"(__uint_as_float(r[4 * c + 1])),
+                             "f"(__uint_as_float(r[4 * c + 2])), "f"(__uint_as_float(r[4 * c + 3]))
+                             : "memory");
+        }
+    }
+}
+
+// ---- MMA issuer ------------------------------------------------------------------
+template <bool BF16>
+__device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars, CtaCtl* ctl)
+{
+    using C = BwdCfg<BF16>;
+    auto bar = [&](int i) { return bars + 8u * i; };
+    const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sDS = base + C::OFF_DS;
+    uint32_t it = 0, unit_it = 0, dq_issued = 0;
+    auto kdesc = [](uint32_t a) { return sdesc_sw128(a, 16, 1024); };
+    auto mdesc = [](uint32_t a) { return sdesc_sw128(a, 16384, 1024); };
+    // S^T (or dP^T) = A B^T over d, both K-major tiles
+    auto mma_kk = [&](uint32_t d_t, uint32_t a, uint32_t b) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+            mma_ss(tmem + d_t, kdesc(a + off), kdesc(b + off), C::IDESC_KK, kk > 0);
+        }
+    };
+    auto wait_dq_free = [&]() -> bool {
+        if (dq_issued == 0) return true;
+        return wait_bar(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_BWD_DQ_EMPTY);
+    };
+    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+        const BwdUnit u = bwd_decode(p, ui);
+        if (u.T == 0) continue;
+        if (!wait_bar(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_BWD_KV_FULL)) return;
+        tc_fence_after();
+        {
+            const int st = it & 1;
+            if (!wait_bar(bar(C::B_Q_FULL + st), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
+            tc_fence_after();
+            mma_kk(C::T_S, sK, base + C::OFF_Q + st * C::TILE);
+            mma_commit(bar(C::B_S_FULL));
+            if (!wait_dq_free()) return;
+            if (!wait_bar(bar(C::B_DO_FULL + st), (it >> 1) & 1u, ctl, W_BWD_DO_FULL)) return;
+            tc_fence_after();
+            mma_kk(C::T_DP, sV, base + C::OFF_DO + st * C::TILE);
+            mma_commit(bar(C::B_DP_FULL));
+        }
+        for (int s = 0; s < u.T; ++s, ++it) {
+            const int st = it & 1;
+            const uint32_t sQ = base + C::OFF_Q + st * C::TILE;
+            const uint32_t sDO = base + C::OFF_DO + st * C::TILE;
+            // dV += P^T dO
+            if (!wait_bar(bar(C::B_P_FULL), it & 1u, ctl, W_BWD_P_FULL)) return;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8, mdesc(sDO + kk * 2048u), C::IDESC_KM,
+                       (s > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar(C::B_DO_EMPTY + st));
+            // next S^T as soon as P^T has been consumed (in-order tensor pipe)
+            const int nst = (it + 1) & 1;
+            if (s + 1 < u.T) {
+                if (!wait_bar(bar(C::B_Q_FULL + nst), ((it + 1) >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
+                tc_fence_after();
+                mma_kk(C::T_S, sK, base + C::OFF_Q + nst * C::TILE);
+                mma_commit(bar(C::B_S_FULL));
+            }
+            // dK += dS^T Q ; dQ_part = dS K
+            if (!wait_bar(bar(C::B_DS_FULL), it & 1u, ctl, W_BWD_DS_FULL)) return;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t a = sDS + (kk >> 2) * 16384u + (kk & 3) * 32u;
+                mma_ss(tmem + C::T_DK, kdesc(a), mdesc(sQ + kk * 2048u), C::IDESC_KM,
+                       (s > 0 || kk > 0) ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + C::T_DP, mdesc(sDS + kk * 2048u), mdesc(sK + kk * 2048u), C::IDESC_MM,
+                       kk > 0 ? 1u : 0u);
+            mma_commit(bar(C::B_DQ_FULL));
+            ++dq_issued;
+            mma_commit(bar(C::B_Q_EMPTY + st));
+            mma_commit(bar(C::B_DS_EMPTY));
+            // next dP^T once the dQ readers have drained TMEM
+            if (s + 1 < u.T) {
+                if (!wait_dq_free()) return;
+                if (!wait_bar(bar(C::B_DO_FULL + nst), ((it + 1) >> 1) & 1u, ctl, W_BWD_DO_FULL)) return;
+                tc_fence_after();
+                mma_kk(C::T_DP, sV, base + C::OFF_DO + nst * C::TILE);
+                mma_commit(bar(C::B_DP_FULL));
+            }
+        }
+        mma_commit(bar(C::B_KV_EMPTY));
+        mma_commit(bar(C::B_DKV_FINAL));
+        ++unit_it;
+    }
+}
+
+// ---- TMA producer --------------------------------------------------------------------
+template <bool BF16>
+struct BwdLoad {
+    using C = BwdCfg<BF16>;
+    const CUtensorMap *tmQ, *tmK, *tmV, *tmDO;
+    uint32_t base, bars;
+    CtaCtl* ctl;
+    int kv_round = -1;
+    int q_round[2] = {-1, -1};
+    int do_round[2] = {-1, -1};
+
+    __device__ uint32_t bar(int i) const { return bars + 8u * i; }
+    __device__ void tile(uint32_t dst, const CUtensorMap* tm, uint32_t b_, int h, int row, int b)
+    {
+        tma_load_4d(dst, tm, b_, 0, h, row, b);
+        tma_load_4d(dst + 16384u, tm, b_, 64, h, row, b);
+    }
+    __device__ void run(const BwdParams& p)
+    {
+        uint32_t it = 0, unit_it = 0;
+        for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+            const BwdUnit u = bwd_decode(p, ui);
+            if (u.T == 0) continue;
+            if (!wait_bar(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_BWD_KV_EMPTY)) return;
+            mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::TILE);
+            tile(base + C::OFF_K, tmK, bar(C::B_KV_FULL), u.hkv, u.n * 128, u.b);
+            tile(base + C::OFF_V, tmV, bar(C::B_KV_FULL), u.hkv, u.n * 128, u.b);
+            kv_round = static_cast<int>(unit_it);
+            ++unit_it;
+            for (int s = 0; s < u.T; ++s, ++it) {
+                int h, m;
+                bwd_step(p, u, s, h, m);
+                const int st = it & 1;
+                const uint32_t ph = ((it >> 1) & 1u) ^ 1u;
+                if (!wait_bar(bar(C::B_Q_EMPTY + st), ph, ctl, W_BWD_Q_EMPTY)) return;
+                mbar_arrive_expect_tx(bar(C::B_Q_FULL + st), C::TILE);
+                tile(base + C::OFF_Q + st * C::TILE, tmQ, bar(C::B_Q_FULL + st), h, m * 128, u.b);
+                q_round[st] = static_cast<int>(it >> 1);
+                if (!wait_bar(bar(C::B_DO_EMPTY + st), ph, ctl, W_BWD_DO_EMPTY)) return;
+                mbar_arrive_expect_tx(bar(C::B_DO_FULL + st), C::TILE);
+                tile(base + C::OFF_DO + st * C::TILE, tmDO, bar(C::B_DO_FULL + st), h, m * 128, u.b);
+                do_round[st] = static_cast<int>(it >> 1);
+            }
+        }
+    }
+    __device__ void drain()
+    {
+        if (kv_round >= 0) drain_wait(bar(C::B_KV_FULL), static_cast<uint32_t>(kv_round) & 1u, W_BWD_DRAIN);
+        for (int st = 0; st < 2; ++st) {
+            if (q_round[st] >= 0) drain_wait(bar(C::B_Q_FULL + st), static_cast<uint32_t>(q_round[st]) & 1u, W_BWD_DRAIN);
+            if (do_round[st] >= 0) drain_wait(bar(C::B_DO_FULL + st), static_cast<uint32_t>(do_round[st]) & 1u, W_BWD_DRAIN);
+        }
+    }
+};
+
+template <bool BF16>
+__global__ void __launch_bounds__(BwdCfg<BF16>::THREADS, 1)
+    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                       const BwdParams p)
+{
+    using C = BwdCfg<BF16>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* base_ptr = smem_raw + (base - raw);
+    const uint32_t bars = base + C::OFF_BAR;
+    CtaCtl* ctl = reinterpret_cast<CtaCtl*>(base_ptr + C::OFF_CTL);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        auto bar = [&](int i) { return bars + 8u * i; };
+        mbar_init(bar(C::B_KV_FULL), 1);
+        mbar_init(bar(C::B_KV_EMPTY), 1);
+        for (int st = 0; st < 2; ++st) {
+            mbar_init(bar(C::B_Q_FULL + st), 1);
+            mbar_init(bar(C::B_Q_EMPTY + st), 1);
+            mbar_init(bar(C::B_DO_FULL + st), 1);
+            mbar_init(bar(C::B_DO_EMPTY + st), 1);
+        }
+        mbar_init(bar(C::B_S_FULL), 1);
+        mbar_init(bar(C::B_DP_FULL), 1);
+        mbar_init(bar(C::B_P_FULL), 4);
+        mbar_init(bar(C::B_DS_FULL), 4);
+        mbar_init(bar(C::B_DS_EMPTY), 1);
+        mbar_init(bar(C::B_DQ_FULL), 1);
+        mbar_init(bar(C::B_DQ_EMPTY), 4);
+        mbar_init(bar(C::B_DKV_FINAL), 1);
+        mbar_init(bar(C::B_DRAIN), 1);
+        ctl->abort = 0u;
+        fence_mbar_init();
+    }
+    if (warp == C::MMA_WARP) {
+        tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+        tmem_relinquish();
+    }
+    if (warp == C::LOAD_WARP && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmDO);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp < 4) {
+        bwd_compute<BF16>(p, tmem, base + C::OFF_DS, bars, ctl, warp);
+    } else if (warp < 8) {
+        bwd_dq_reduce<BF16>(p, tmem, bars, ctl, warp - 4);
+    } else if (warp == C::MMA_WARP) {
+        if (lane == 0) {
+            bwd_mma<BF16>(p, tmem, base, bars, ctl);
+            mma_commit(bars + 8u * C::B_DRAIN);
+            drain_wait(bars + 8u * C::B_DRAIN, 0u, W_BWD_DRAIN);
+        }
+        __syncwarp();
+    } else if (warp == C::LOAD_WARP) {
+        if (lane == 0) {
+            BwdLoad<BF16> ld{&tmQ, &tmK, &tmV, &tmDO, base, bars, ctl};
+            ld.run(p);
+            ld.drain();
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == C::MMA_WARP) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace fa
