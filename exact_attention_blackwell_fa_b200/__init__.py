@@ -7,6 +7,7 @@ library's CUDA kernels.  The functions carry the C names:
     fa_fwd(q, k, v, causal=False, scale=None) -> (o, lse)
     fa_bwd(q, k, v, o, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
     fa_bwd_workspace_size(B, Sq, Hq, d) -> int
+    fa_bwd_noalloc(q, k, v, o, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
     fa_status_string(code) -> str
     fa_last_device_status() -> (code, detail)
     fa_clear_device_status()
@@ -25,7 +26,7 @@ import torch
 from . import _lib
 
 __all__ = [
-    "FAError", "fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_status_string",
+    "FAError", "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
     "fa_last_device_status", "fa_clear_device_status", "fa_debug_inject",
 ]
 
@@ -119,6 +120,31 @@ def fa_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = No
                               float(scale), _dtype_code(q), workspace.data_ptr(),
                               workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _raise(code, "fa_bwd")
+    return dq, dk, dv
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+                   dq=None, dk=None, dv=None, stream=None):
+    """Backward without a workspace: the library keeps the scratch in a fixed device
+    array (for callers that cannot allocate device memory).  Calls that overlap on
+    the GPU race on that array.  Output tensors may be passed in to avoid allocating
+    them here too.  Returns (dq, dk, dv)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check(t, name, q.dtype)
+    _check(lse, "lse", torch.float32)
+    B, Sq, Hq, d = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    code = _lib.load().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      lse.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+                                      dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, Hq, Hkv, d,
+                                      int(bool(causal)), float(scale), _dtype_code(q),
+                                      _stream_ptr(stream))
+    _raise(code, "fa_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -8,7 +8,9 @@ import threading
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa.so")
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT = range(5)
+(FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT,
+ FA_ERR_SCRATCH_LIMIT) = range(6)
+FA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 FA_BF16, FA_FP16 = 0, 1
 
 # Every symbol include/fa.h declares, with its ctypes signature.
@@ -21,6 +23,8 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (_sz, [_ci, _ci, _ci, _ci]),
     "fa_bwd": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci,
                      _ci, _cf, _ci, _vp, _sz, _vp]),
+    "fa_bwd_noalloc": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
+                             _ci, _ci, _ci, _cf, _ci, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_ci]),
     "fa_last_device_status": (_ci, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "fa_clear_device_status": (_ci, [_vp]),

@@ -277,6 +277,8 @@ const char* fa_status_string(fa_status s)
     case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: head_dim, dtype or GPU not supported";
     case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
     case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
+    case FA_ERR_SCRATCH_LIMIT:
+        return "FA_ERR_SCRATCH_LIMIT: problem needs more scratch than fa_bwd_noalloc's built-in array";
     }
     return "unknown fa_status";
 }
@@ -311,3 +313,50 @@ fa_status fa_debug_inject(int mode)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// fa_bwd_noalloc: fa_bwd with its scratch in a fixed device array, for callers that
+// cannot allocate device memory (a caller-owned pool or arena that forbids
+// cudaMalloc, loops that cannot afford the synchronisation cudaMalloc/cudaFree imply,
+// an embedded host without a device allocator of its own).  Every call on a device
+// shares the array; calls whose kernels overlap on the GPU race on it.
+// ---------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_noalloc_scratch, looked up once per device.  In host code the
+// array's name is only a host-side stand-in, so kernels must be given this address.
+fa_status noalloc_scratch(void** out)
+{
+    static void* addr[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return FA_ERR_CUDA;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                    const float* lse, const void* dout, void* dq, void* dk,
+                                    void* dv, int B, int Sq, int Sk, int Hq, int Hkv, int d,
+                                    int causal, float scale, fa_dtype dt, fa_stream stream)
+{
+    fa_status st = check_common(B, Sq, Sk, Hq, Hkv, d, scale, dt);
+    if (st != FA_OK) return st;
+    if (fa::bwd_workspace_bytes(B, Sq, Hq, d) > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_SCRATCH_LIMIT;
+    void* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != FA_OK) return st;
+    return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Sq, Sk, Hq, Hkv, d, causal, scale, dt,
+                  scratch, FA_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -48,7 +48,8 @@ typedef enum {
     FA_ERR_INVALID_ARG = 1,    /* a size, pointer, alignment or scale is invalid          */
     FA_ERR_UNSUPPORTED = 2,    /* head_dim, dtype or GPU architecture not supported       */
     FA_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed                       */
-    FA_ERR_DEVICE_TIMEOUT = 4  /* a kernel gave up on a bounded wait (see status query)   */
+    FA_ERR_DEVICE_TIMEOUT = 4, /* a kernel gave up on a bounded wait (see status query)   */
+    FA_ERR_SCRATCH_LIMIT = 5   /* problem needs more than the built-in scratch array      */
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
@@ -82,6 +83,36 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  const void* dout, void* dq, void* dk, void* dv,
                  int B, int Sq, int Sk, int Hq, int Hkv, int d, int causal, float scale,
                  fa_dtype dt, void* workspace, size_t workspace_bytes, fa_stream stream);
+
+/*
+ * Backward that allocates nothing and takes no workspace: the same computation as
+ * fa_bwd, with its scratch (the row terms and the float32 dQ accumulator) kept in a
+ * fixed device array built into the library.  The paper has no counterpart to this
+ * entry point; it exists for callers that cannot allocate device memory: code that
+ * runs under a caller-owned memory pool or arena which forbids cudaMalloc, latency-
+ * critical loops that cannot afford the device-wide synchronisation cudaMalloc and
+ * cudaFree imply, and embedded hosts without a device allocator of their own.
+ *
+ * Limit: the scratch array is FA_NOALLOC_SCRATCH_BYTES (32 MiB) on every device
+ * that loads the library, held until the process exits.  A problem whose
+ * fa_bwd_workspace_size(B, Sq, Hq, d) exceeds it returns FA_ERR_SCRATCH_LIMIT and
+ * launches nothing (for d = 128 that is B * Hq * ceil(Sq / 128) * 128 > 64,527
+ * query rows in total).
+ *
+ * Set-up: the first call on each device looks up the device address of the array
+ * (with that device current); make that first call before any stream capture.
+ * Every call on a device shares the one array and leaves its contents behind; the
+ * kernels rewrite everything they read from it (the accumulator is zeroed by the
+ * first kernel of each call), but two calls whose kernels overlap on the GPU --
+ * on different streams, or from different host threads -- race on it.  Serialise
+ * them.  Arguments, layouts and the other errors are as for fa_bwd.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                         int B, int Sq, int Sk, int Hq, int Hkv, int d, int causal, float scale,
+                         fa_dtype dt, fa_stream stream);
 
 /* Static, human-readable name of a status code. */
 const char* fa_status_string(fa_status s);
