@@ -11,6 +11,7 @@
 
 #include "../../include/fa.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd256.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -35,16 +36,17 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 4-D map over a [B, S, H, d] 16-bit tensor; one box = 64 head-dim columns x 128 rows
-// of one (batch, head), 128-byte swizzled.  Rows past S read as zero.
-bool make_tmap(CUtensorMap* m, const void* ptr, int B, int S, int H, int d, bool bf16)
+// 4-D map over a [B, S, H, d] 16-bit tensor; one box = 64 head-dim columns x box_rows
+// rows of one (batch, head), 128-byte swizzled.  Rows past S read as zero.
+bool make_tmap(CUtensorMap* m, const void* ptr, int B, int S, int H, int d, bool bf16,
+               int box_rows = 128)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
                                    (cuuint64_t)S * H * d * 2};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
                const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -144,6 +146,25 @@ fa_status launch_bwd_d128(const CUtensorMap& tq, const CUtensorMap& tk, const CU
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+template <bool BF16>
+fa_status launch_bwd_d256(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64,
+                          const CUtensorMap& tdo, const fa::BwdParams& p, int sm_count,
+                          cudaStream_t stream)
+{
+    using C = fa::Bwd256Cfg<BF16>;
+    const long long pre_rows = (long long)p.B * p.Hq * p.Sq_pad;
+    fa::fa_bwd_pre_kernel<256, BF16><<<(unsigned)((pre_rows + 7) / 8), 256, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    fa_status st = set_smem(fa::fa_bwd_dkdv256_kernel<BF16>, C::SMEM_BYTES);
+    if (st != FA_OK) return st;
+    const int grid = p.num_units < sm_count ? p.num_units : sm_count;
+    fa::fa_bwd_dkdv256_kernel<BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk64, tv64, tdo, p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    const long long dq_rows = (long long)p.B * p.Sq * p.Hq;
+    fa::fa_bwd_dq_kernel<256, BF16><<<(unsigned)((dq_rows + 7) / 8), 256, 0, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 template <int D, bool BF16>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      fa::FwdParams p, int sm_count, cudaStream_t stream)
@@ -151,6 +172,7 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
     using C = fa::FwdCfg<D, BF16>;
     fa_status st = set_smem(fa::fa_fwd_kernel<D, BF16>, C::SMEM_BYTES);
     if (st != FA_OK) return st;
+
     const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
     fa::fa_fwd_kernel<D, BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -224,11 +246,11 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     DeviceInfo di;
     st = device_info(&di);
     if (st != FA_OK) return st;
-    if (d != 128) return FA_ERR_UNSUPPORTED;
     const bool bf16 = dt == FA_BF16;
+    const int kv_rows = d == 128 ? 128 : 64;  // keys per backward work unit
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_tmap(&tq, q, B, Sq, Hq, d, bf16) || !make_tmap(&tk, k, B, Sk, Hkv, d, bf16) ||
-        !make_tmap(&tv, v, B, Sk, Hkv, d, bf16) || !make_tmap(&tdo, dout, B, Sq, Hq, d, bf16))
+    if (!make_tmap(&tq, q, B, Sq, Hq, d, bf16) || !make_tmap(&tk, k, B, Sk, Hkv, d, bf16, kv_rows) ||
+        !make_tmap(&tv, v, B, Sk, Hkv, d, bf16, kv_rows) || !make_tmap(&tdo, dout, B, Sq, Hq, d, bf16))
         return FA_ERR_CUDA;
     fa::BwdParams p{};
     p.o = o;
@@ -250,7 +272,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     p.Hkv = Hkv;
     p.group = Hq / Hkv;
     p.Sq_pad = (int)sq_pad;
-    p.num_n = (Sk + 127) / 128;
+    p.num_n = (Sk + kv_rows - 1) / kv_rows;
     p.num_m = (Sq + 127) / 128;
     p.num_units = B * Hkv * p.num_n;
     // KV heads whose Q and dO streams stay inside L2 together
@@ -265,6 +287,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     p.scale = scale;
     p.sl2 = scale * 1.4426950408889634f;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 256)
+        return bf16 ? launch_bwd_d256<true>(tq, tk, tv, tdo, p, di.sm_count, s)
+                    : launch_bwd_d256<false>(tq, tk, tv, tdo, p, di.sm_count, s);
     return bf16 ? launch_bwd_d128<true>(tq, tk, tv, tdo, p, di.sm_count, s)
                 : launch_bwd_d128<false>(tq, tk, tv, tdo, p, di.sm_count, s);
 }

@@ -62,7 +62,7 @@ struct BwdParams {
 enum : uint32_t {
     W_BWD_KV_FULL = 0x201, W_BWD_KV_EMPTY, W_BWD_Q_FULL, W_BWD_Q_EMPTY, W_BWD_DO_FULL,
     W_BWD_DO_EMPTY, W_BWD_S_FULL, W_BWD_DP_FULL, W_BWD_P_FULL, W_BWD_DS_FULL, W_BWD_DS_EMPTY,
-    W_BWD_DQ_FULL, W_BWD_DQ_EMPTY, W_BWD_DKV_FINAL, W_BWD_DRAIN
+    W_BWD_DQ_FULL, W_BWD_DQ_EMPTY, W_BWD_DKV_FINAL, W_BWD_DRAIN, W_BWD_SMEM_ALIGN
 };
 
 // ---------------------------------------------------------------------------------
@@ -155,14 +155,20 @@ struct BwdCfg {
     static constexpr int THREADS = 384;
     static constexpr int MMA_WARP = 8, LOAD_WARP = 9;
     static constexpr uint32_t TILE = 32768;  // 128 rows x 128 columns x 2 bytes
+    // per query block: LSE*log2(e) and D for its 128 rows, staged with the Q tile
+    static constexpr uint32_t ROWS_BYTES = 1024;
     static constexpr uint32_t OFF_K = 0, OFF_V = TILE, OFF_Q = 2 * TILE, OFF_DO = 4 * TILE,
-                              OFF_DS = 6 * TILE, OFF_BAR = 7 * TILE;
+                              OFF_DS = 6 * TILE, OFF_ROWS = 7 * TILE,
+                              OFF_BAR = OFF_ROWS + 2 * ROWS_BYTES;
     static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1, B_Q_FULL = 2, B_Q_EMPTY = 4, B_DO_FULL = 6,
                          B_DO_EMPTY = 8, B_S_FULL = 10, B_DP_FULL = 11, B_P_FULL = 12, B_DS_FULL = 13,
                          B_DS_EMPTY = 14, B_DQ_FULL = 15, B_DQ_EMPTY = 16, B_DKV_FINAL = 17,
                          B_DRAIN = 18, NBAR = 19;
     static constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
-    static constexpr uint32_t SMEM_BYTES = OFF_CTL + sizeof(CtaCtl) + 1024;
+    // no alignment slack: the dynamic shared memory base must be 1024-byte aligned,
+    // which the kernel checks before it touches anything
+    static constexpr uint32_t SMEM_BYTES = OFF_CTL + sizeof(CtaCtl);
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     // TMEM columns
     static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
     static constexpr uint32_t IDESC_KK = idesc_f16(BF16, 128, 128, false, false);  // S^T, dP^T
@@ -210,15 +216,17 @@ __device__ __forceinline__ void bwd_step(const BwdParams& p, const BwdUnit& u, i
 
 // ---- compute warpgroup: P^T and dS^T, then the dK / dV epilogue --------------------
 template <bool BF16>
-__device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uint32_t bars,
-                            CtaCtl* ctl, int wq)
+__device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uint32_t sRows,
+                            uint32_t bars, CtaCtl* ctl, int wq)
 {
     using C = BwdCfg<BF16>;
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
     const int lane = threadIdx.x & 31;
     const int t = wq * 32 + lane;  // key row within the block (= TMEM lane)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::T_S, tDP = tmem + lane_off + C::T_DP;
     auto bar = [&](int i) { return bars + 8u * i; };
+    const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
     uint32_t it = 0, unit_it = 0;
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
         const BwdUnit u = bwd_decode(p, ui);
@@ -226,71 +234,93 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
         for (int s = 0; s < u.T; ++s, ++it) {
             int h, m;
             bwd_step(p, u, s, h, m);
-            const size_t rbase = (static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + static_cast<size_t>(m) * 128;
-            const float4* L2v = reinterpret_cast<const float4*>(p.L2 + rbase);
-            const float4* Dvv = reinterpret_cast<const float4*>(p.Dv + rbase);
+            const uint32_t rows = sRows + (it & 1) * C::ROWS_BYTES;  // L2[128] then D[128]
             // key j is visible to query i iff j <= i + (Sk - Sq)
             const bool masked = p.causal && (u.n * 128 + 127 > m * 128 + p.Sk - p.Sq);
             const int jlim = j - (p.Sk - p.Sq) - m * 128;  // visible iff column c >= jlim
+            // the Q-tile barrier also covers the staged row terms
+            if (!warp_wait(bar(C::B_Q_FULL + (it & 1)), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
             if (!warp_wait(bar(C::B_S_FULL), it & 1u, ctl, W_BWD_S_FULL)) return;
             tc_fence_after();
-            float P[128];
+            // P^T = 2^(S^T scale log2e - LSE log2e), 32 query columns at a time.  The
+            // 16-bit P^T words stay in registers for dS: the MMA issues the next S^T into
+            // these TMEM columns as soon as dV has consumed them.
+            uint32_t ppk[64];
+            uint32_t rbuf[2][32];
+            tmem_ld32_nowait(tS, rbuf[0]);
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-                uint32_t r[32];
-                tmem_ld32_wait(tmem + lane_off + C::T_S + cc * 32, r);
-                uint32_t pk[16];
+                uint32_t (&r)[32] = rbuf[cc & 1];
+                tmem_wait_ld_dep(r);
+                if (cc + 1 < 4) tmem_ld32_nowait(tS + (cc + 1) * 32, rbuf[(cc + 1) & 1]);
+                uint32_t (&pk)[16] = *reinterpret_cast<uint32_t(*)[16]>(&ppk[cc * 16]);
 #pragma unroll
                 for (int k4 = 0; k4 < 8; ++k4) {
-                    const float4 l4 = L2v[cc * 8 + k4];
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    float4 l4;
+                    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                 : "=f"(l4.x), "=f"(l4.y), "=f"(l4.z), "=f"(l4.w)
+                                 : "r"(rows + (cc * 32 + k4 * 4) * 4u));
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = cc * 32 + k4 * 4 + e;
-                        const float x = fmaf(__uint_as_float(r[k4 * 4 + e]), p.sl2, -lv[e]);
-                        float pv = ((e & 1) && !masked) ? exp2_fma(x) : ex2_sfu(x);
-                        if (masked && c < jlim) pv = 0.0f;
-                        P[c] = pv;
+                    for (int e = 0; e < 4; e += 2) {
+                        const int k = k4 * 4 + e;
+                        const float la = e == 0 ? l4.x : l4.z, lb = e == 0 ? l4.y : l4.w;
+                        const float2 x = f2unpack(ffma2(f2pack(__uint_as_float(r[k]), __uint_as_float(r[k + 1])),
+                                                        sl2x2, f2pack(-la, -lb)));
+                        float e0, e1;
+                        if (!masked && (k & 2)) {
+                            exp2_fma_x2(x.x, x.y, e0, e1);
+                        } else {
+                            e0 = ex2_sfu(x.x);
+                            e1 = ex2_sfu(x.y);
+                        }
+                        if (masked) {
+                            const int c = cc * 32 + k;
+                            if (c < jlim) e0 = 0.0f;
+                            if (c + 1 < jlim) e1 = 0.0f;
+                        }
+                        pk[k >> 1] = pack2<BF16>(e0, e1);
                     }
                 }
-#pragma unroll
-                for (int k = 0; k < 16; ++k) pk[k] = pack2<BF16>(P[cc * 32 + 2 * k], P[cc * 32 + 2 * k + 1]);
-                tmem_st16(tmem + lane_off + C::T_S + cc * 16, pk);
+                tmem_st16(tS + cc * 16, pk);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_P_FULL));
 
+            // dS^T = P^T (dP^T - D), 32 query columns at a time (next chunk's load in flight)
             if (!warp_wait(bar(C::B_DP_FULL), it & 1u, ctl, W_BWD_DP_FULL)) return;
             if (!warp_wait(bar(C::B_DS_EMPTY), (it & 1u) ^ 1u, ctl, W_BWD_DS_EMPTY)) return;
             tc_fence_after();
+            tmem_ld32_nowait(tDP, rbuf[0]);
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-                uint32_t r[32];
-                tmem_ld32_wait(tmem + lane_off + C::T_DP + cc * 32, r);
-                uint32_t pk[16];
+                uint32_t (&r)[32] = rbuf[cc & 1];
+                tmem_wait_ld_dep(r);
+                if (cc + 1 < 4) tmem_ld32_nowait(tDP + (cc + 1) * 32, rbuf[(cc + 1) & 1]);
 #pragma unroll
-                for (int k4 = 0; k4 < 8; ++k4) {
-                    const float4 d4 = Dvv[cc * 8 + k4];
-                    const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float ds[4];
+                for (int g = 0; g < 4; ++g) {  // 8 query columns -> one 16-byte chunk
+                    float4 da, db;
+                    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                 : "=f"(da.x), "=f"(da.y), "=f"(da.z), "=f"(da.w)
+                                 : "r"(rows + 512u + (cc * 32 + g * 8) * 4u));
+                    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                 : "=f"(db.x), "=f"(db.y), "=f"(db.z), "=f"(db.w)
+                                 : "r"(rows + 512u + (cc * 32 + g * 8 + 4) * 4u));
+                    const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+                    uint32_t q4[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = cc * 32 + k4 * 4 + e;
-                        ds[e] = P[c] * (__uint_as_float(r[k4 * 4 + e]) - dv[e]);
+                    for (int w = 0; w < 4; ++w) {
+                        const int k = g * 8 + w * 2;  // column within the chunk
+                        const float2 pp = unpack2<BF16>(ppk[cc * 16 + (k >> 1)]);
+                        q4[w] = pack2<BF16>(pp.x * (__uint_as_float(r[k]) - dv[w * 2]),
+                                            pp.y * (__uint_as_float(r[k + 1]) - dv[w * 2 + 1]));
                     }
-                    pk[k4 * 2] = pack2<BF16>(ds[0], ds[1]);
-                    pk[k4 * 2 + 1] = pack2<BF16>(ds[2], ds[3]);
-                }
-                // columns cc*32 .. cc*32+31 = four 16-byte chunks of row t, 128-byte swizzle
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
                     const int col8 = cc * 4 + g;  // 8-column group 0..15
                     const uint32_t addr = sDS + (col8 >> 3) * 16384u + t * 128u +
                                           ((static_cast<uint32_t>(col8 & 7) ^ (t & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                                 "r"(pk[4 * g]), "r"(pk[4 * g + 1]), "r"(pk[4 * g + 2]), "r"(pk[4 * g + 3])
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(q4[0]),
+                                 "r"(q4[1]), "r"(q4[2]), "r"(q4[3])
                                  : "memory");
                 }
             }
@@ -492,8 +522,15 @@ struct BwdLoad {
                 const int st = it & 1;
                 const uint32_t ph = ((it >> 1) & 1u) ^ 1u;
                 if (!wait_bar(bar(C::B_Q_EMPTY + st), ph, ctl, W_BWD_Q_EMPTY)) return;
-                mbar_arrive_expect_tx(bar(C::B_Q_FULL + st), C::TILE);
+                mbar_arrive_expect_tx(bar(C::B_Q_FULL + st), C::TILE + C::ROWS_BYTES);
                 tile(base + C::OFF_Q + st * C::TILE, tmQ, bar(C::B_Q_FULL + st), h, m * 128, u.b);
+                {
+                    const size_t rb = (static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad +
+                                      static_cast<size_t>(m) * 128;
+                    const uint32_t dst = base + C::OFF_ROWS + st * C::ROWS_BYTES;
+                    bulk_load(dst, p.L2 + rb, 512, bar(C::B_Q_FULL + st));
+                    bulk_load(dst + 512, p.Dv + rb, 512, bar(C::B_Q_FULL + st));
+                }
                 q_round[st] = static_cast<int>(it >> 1);
                 if (!wait_bar(bar(C::B_DO_EMPTY + st), ph, ctl, W_BWD_DO_EMPTY)) return;
                 mbar_arrive_expect_tx(bar(C::B_DO_FULL + st), C::TILE);
@@ -520,11 +557,15 @@ __global__ void __launch_bounds__(BwdCfg<BF16>::THREADS, 1)
 {
     using C = BwdCfg<BF16>;
     extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* base_ptr = smem_raw + (base - raw);
+    const uint32_t base = smem_u32(smem_raw);
+    if (base & 1023u) {  // swizzled TMA tiles and MMA descriptors need 1024-byte alignment
+        if (threadIdx.x == 0 &&
+            atomicCAS(&g_status[0], 0u, static_cast<uint32_t>(FA_ERR_UNSUPPORTED)) == 0u)
+            g_status[1] = W_BWD_SMEM_ALIGN;
+        return;
+    }
     const uint32_t bars = base + C::OFF_BAR;
-    CtaCtl* ctl = reinterpret_cast<CtaCtl*>(base_ptr + C::OFF_CTL);
+    CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem_raw + C::OFF_CTL);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -565,7 +606,7 @@ __global__ void __launch_bounds__(BwdCfg<BF16>::THREADS, 1)
     const uint32_t tmem = ctl->tmem_base;
 
     if (warp < 4) {
-        bwd_compute<BF16>(p, tmem, base + C::OFF_DS, bars, ctl, warp);
+        bwd_compute<BF16>(p, tmem, base + C::OFF_DS, base + C::OFF_ROWS, bars, ctl, warp);
     } else if (warp < 8) {
         bwd_dq_reduce<BF16>(p, tmem, bars, ctl, warp - 4);
     } else if (warp == C::MMA_WARP) {

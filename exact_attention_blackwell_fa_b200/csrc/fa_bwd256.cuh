@@ -1,0 +1,471 @@
+// fa_bwd256.cuh -- dK / dV / dQ-partials kernel of the attention backward for head_dim 256.
+//
+// Same arithmetic as the head_dim 128 kernel in fa_bwd.cuh (P recomputed from LSE,
+// dS = P (dP - D), dV = P^T dO, dK = scale dS^T Q, dQ partials reduced in fp32), with
+// a tiling that fits 256-wide heads into 512 TMEM columns and 227 KB of shared memory:
+//
+//   * a work unit is 64 keys of one (batch, KV head); it loops over the group's query
+//     heads and 128-row query blocks;
+//   * S = Q K^T and dP = dO V^T are computed query-major (M = 128 query rows, N = 64
+//     keys), so the compute warpgroup's thread owns one query row and its LSE and D;
+//   * P and dS go to shared memory as [query][key] tiles (128-byte swizzle); the
+//     key-side accumulators are kept transposed, dV^T += dO^T P and dK^T += Q^T dS,
+//     as two M = 128 head-dim halves each, reading dO, Q (MN-major) and P, dS
+//     (MN-major) straight from the tiles already in shared memory;
+//   * dQ = dS K is produced in two 128-column halves into one TMEM region, each drained
+//     by the dQ warpgroup into the fp32 accumulator with vector reductions.
+//
+// TMEM: S [0,64) | dP [64,128) | dQ half [128,256) | dV^T halves [256,384) | dK^T [384,512)
+#pragma once
+
+#include "fa_bwd.cuh"
+
+namespace fa {
+
+template <bool BF16>
+struct Bwd256Cfg {
+    static constexpr int D = 256;
+    static constexpr int BN = 64;   // keys per unit
+    static constexpr int BM = 128;  // query rows per step
+    static constexpr int THREADS = 384;
+    static constexpr int MMA_WARP = 8, LOAD_WARP = 9;
+    static constexpr uint32_t KV_BLK = BN * 128;   // [64 rows][64 cols] of 16-bit values
+    static constexpr uint32_t KV_BYTES = 4 * KV_BLK;
+    static constexpr uint32_t Q_BLK = BM * 128;    // [128 rows][64 cols]
+    static constexpr uint32_t Q_BYTES = 4 * Q_BLK;
+    static constexpr uint32_t PT_BYTES = BM * BN * 2;  // [128 queries][64 keys]
+    static constexpr uint32_t ROWS_BYTES = 1024;       // LSE*log2(e)[128], D[128]
+    static constexpr uint32_t OFF_K = 0, OFF_V = KV_BYTES, OFF_Q = 2 * KV_BYTES,
+                              OFF_DO = OFF_Q + Q_BYTES, OFF_P = OFF_DO + Q_BYTES,
+                              OFF_DS = OFF_P + PT_BYTES, OFF_ROWS = OFF_DS + PT_BYTES,
+                              OFF_BAR = OFF_ROWS + ROWS_BYTES;
+    static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1, B_Q_FULL = 2, B_Q_EMPTY = 3, B_DO_FULL = 4,
+                         B_DO_EMPTY = 5, B_S_FULL = 6, B_DP_FULL = 7, B_P_FULL = 8, B_P_EMPTY = 9,
+                         B_DS_FULL = 10, B_DS_EMPTY = 11, B_DQ_FULL = 12, B_DQ_EMPTY = 13,
+                         B_DKV_FINAL = 14, B_DRAIN = 15, NBAR = 16;
+    static constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
+    static constexpr uint32_t SMEM_BYTES = OFF_CTL + sizeof(CtaCtl);
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static constexpr uint32_t T_S = 0, T_DP = 64, T_DQ = 128, T_DV = 256, T_DK = 384;
+    static constexpr uint32_t IDESC_S = idesc_f16(BF16, 128, 64, false, false);   // S, dP
+    static constexpr uint32_t IDESC_T = idesc_f16(BF16, 128, 64, true, true);     // dV^T, dK^T
+    static constexpr uint32_t IDESC_Q = idesc_f16(BF16, 128, 128, false, true);   // dQ half
+};
+
+enum : uint32_t {
+    W_B256_KV_FULL = 0x301, W_B256_KV_EMPTY, W_B256_Q_FULL, W_B256_Q_EMPTY, W_B256_DO_FULL,
+    W_B256_DO_EMPTY, W_B256_S_FULL, W_B256_DP_FULL, W_B256_P_FULL, W_B256_P_EMPTY,
+    W_B256_DS_FULL, W_B256_DS_EMPTY, W_B256_DQ_FULL, W_B256_DQ_EMPTY, W_B256_DKV_FINAL,
+    W_B256_DRAIN, W_B256_SMEM_ALIGN
+};
+
+// num_n counts 64-key blocks here
+__device__ __forceinline__ BwdUnit bwd256_decode(const BwdParams& p, int t)
+{
+    const int BH = p.B * p.Hkv;
+    const int per_chunk = p.chunk_heads * p.num_n;
+    const int c = t / per_chunk;
+    const int r = t - c * per_chunk;
+    const int first = c * p.chunk_heads;
+    const int csize = min(p.chunk_heads, BH - first);
+    const int nb = r / csize;  // causal: ascending key block = most query blocks first
+    const int bh = first + (r - nb * csize);
+    BwdUnit u;
+    u.b = bh / p.Hkv;
+    u.hkv = bh - u.b * p.Hkv;
+    u.n = nb;
+    int ms = 0;
+    if (p.causal) {
+        const long long imin = static_cast<long long>(u.n) * 64 - (p.Sk - p.Sq);
+        ms = imin <= 0 ? 0 : static_cast<int>(imin / 128);
+        if (ms > p.num_m) ms = p.num_m;
+    }
+    u.m_start = ms;
+    u.nm = p.num_m - ms;
+    u.T = p.group * u.nm;
+    return u;
+}
+
+// P or dS row of one query (64 keys, 16-bit) into a [128][64] tile, 128-byte swizzle
+__device__ __forceinline__ void store_tile_row(uint32_t tile, int row, const uint32_t (&w)[32])
+{
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+        const uint32_t addr = tile + row * 128u + ((static_cast<uint32_t>(c8) ^ (row & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * c8]),
+                     "r"(w[4 * c8 + 1]), "r"(w[4 * c8 + 2]), "r"(w[4 * c8 + 3])
+                     : "memory");
+    }
+}
+
+// ---- compute warpgroup (thread = query row): P and dS; then the dV / dK epilogue ----
+template <bool BF16>
+__device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars,
+                               CtaCtl* ctl, int wq)
+{
+    using C = Bwd256Cfg<BF16>;
+    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    const int lane = threadIdx.x & 31;
+    const int t = wq * 32 + lane;  // query row within the block, and head-dim lane later
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    auto bar = [&](int i) { return bars + 8u * i; };
+    const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
+    uint32_t it = 0, unit_it = 0;
+    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+        const BwdUnit u = bwd256_decode(p, ui);
+        for (int s = 0; s < u.T; ++s, ++it) {
+            int h, m;
+            bwd_step(p, u, s, h, m);
+            const int i = m * 128 + t;  // query row
+            // key n*64 + c is visible iff c <= lim
+            const int lim = i + (p.Sk - p.Sq) - u.n * 64;
+            const bool masked = p.causal && (u.n * 64 + 63 > m * 128 + p.Sk - p.Sq);
+            if (!warp_wait(bar(C::B_Q_FULL), it & 1u, ctl, W_B256_Q_FULL)) return;
+            float l2, dval;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l2) : "r"(base + C::OFF_ROWS + t * 4u));
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dval) : "r"(base + C::OFF_ROWS + 512u + t * 4u));
+            const uint64_t negl2 = f2pack(-l2, -l2);
+            if (!warp_wait(bar(C::B_S_FULL), it & 1u, ctl, W_B256_S_FULL)) return;
+            tc_fence_after();
+            uint32_t r0[32], r1[32];
+            tmem_ld32_nowait(tmem + lane_off + C::T_S, r0);
+            tmem_ld32_nowait(tmem + lane_off + C::T_S + 32, r1);
+            tmem_wait_ld_dep(r0);
+            tmem_wait_ld_dep(r1);
+            float P[64];
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+                const uint32_t a = c < 32 ? r0[c] : r1[c - 32];
+                const uint32_t b = c < 32 ? r0[c + 1] : r1[c - 31];
+                const float2 x = f2unpack(ffma2(f2pack(__uint_as_float(a), __uint_as_float(b)), sl2x2, negl2));
+                float e0, e1;
+                if (!masked && (c & 2)) {
+                    exp2_fma_x2(x.x, x.y, e0, e1);
+                } else {
+                    e0 = ex2_sfu(x.x);
+                    e1 = ex2_sfu(x.y);
+                }
+                if (masked) {
+                    if (c > lim) e0 = 0.0f;
+                    if (c + 1 > lim) e1 = 0.0f;
+                }
+                P[c] = e0;
+                P[c + 1] = e1;
+            }
+            {
+                uint32_t w[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) w[k] = pack2<BF16>(P[2 * k], P[2 * k + 1]);
+                if (!warp_wait(bar(C::B_P_EMPTY), (it & 1u) ^ 1u, ctl, W_B256_P_EMPTY)) return;
+                store_tile_row(base + C::OFF_P, t, w);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_P_FULL));
+
+            if (!warp_wait(bar(C::B_DP_FULL), it & 1u, ctl, W_B256_DP_FULL)) return;
+            tc_fence_after();
+            tmem_ld32_nowait(tmem + lane_off + C::T_DP, r0);
+            tmem_ld32_nowait(tmem + lane_off + C::T_DP + 32, r1);
+            tmem_wait_ld_dep(r0);
+            tmem_wait_ld_dep(r1);
+            {
+                uint32_t w[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int c = 2 * k;
+                    const uint32_t a = c < 32 ? r0[c] : r1[c - 32];
+                    const uint32_t b = c < 32 ? r0[c + 1] : r1[c - 31];
+                    w[k] = pack2<BF16>(P[c] * (__uint_as_float(a) - dval), P[c + 1] * (__uint_as_float(b) - dval));
+                }
+                if (!warp_wait(bar(C::B_DS_EMPTY), (it & 1u) ^ 1u, ctl, W_B256_DS_EMPTY)) return;
+                store_tile_row(base + C::OFF_DS, t, w);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_DS_FULL));
+        }
+        // epilogue: thread t holds head-dim column (half * 128 + t) of dV^T / dK^T
+        if (!warp_wait(bar(C::B_DKV_FINAL), unit_it & 1u, ctl, W_B256_DKV_FINAL)) return;
+        ++unit_it;
+        tc_fence_after();
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+            const float mul = which == 0 ? 1.0f : p.scale;
+            T* dst = static_cast<T*>(which == 0 ? p.dv : p.dk);
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint32_t col = (which == 0 ? C::T_DV : C::T_DK) + hf * 64;
+                uint32_t r[32];
+#pragma unroll 1
+                for (int cc = 0; cc < 2; ++cc) {
+                    tmem_ld32_wait(tmem + lane_off + col + cc * 32, r);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int key = u.n * 64 + cc * 32 + c;
+                        if (key < p.Sk) {
+                            const size_t off =
+                                ((static_cast<size_t>(u.b) * p.Sk + key) * p.Hkv + u.hkv) * C::D + hf * 128 + t;
+                            dst[off] = static_cast<T>(__uint_as_float(r[c]) * mul);
+                        }
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+    }
+}
+
+// ---- dQ warpgroup: two 128-column halves per step -> fp32 vector reductions ----------
+template <bool BF16>
+__device__ void bwd256_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int wq)
+{
+    using C = Bwd256Cfg<BF16>;
+    const int lane = threadIdx.x & 31;
+    const int t = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    auto bar = [&](int i) { return bars + 8u * i; };
+    uint32_t k = 0;  // dQ halves drained so far
+    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+        const BwdUnit u = bwd256_decode(p, ui);
+        for (int s = 0; s < u.T; ++s) {
+            int h, m;
+            bwd_step(p, u, s, h, m);
+            float* row = p.dqacc + ((static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + m * 128 + t) * C::D;
+#pragma unroll 1
+            for (int dh = 0; dh < 2; ++dh, ++k) {
+                if (!warp_wait(bar(C::B_DQ_FULL), k & 1u, ctl, W_B256_DQ_FULL)) return;
+                tc_fence_after();
+                uint32_t r[128];
+                tmem_ld128_wait(tmem + lane_off + C::T_DQ, r);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
+                float* dst = row + dh * 128;
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * c),
+                                 "f"(__uint_as_float(r[4 * c])), "f"(__uint_as_float(r[4 * c + 1])),
+                                 "f"(__uint_as_float(r[4 * c + 2])), "f"(__uint_as_float(r[4 * c + 3]))
+                                 : "memory");
+            }
+        }
+    }
+}
+
+// ---- MMA issuer ----------------------------------------------------------------------
+template <bool BF16>
+__device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars, CtaCtl* ctl)
+{
+    using C = Bwd256Cfg<BF16>;
+    auto bar = [&](int i) { return bars + 8u * i; };
+    const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQ = base + C::OFF_Q,
+                   sDO = base + C::OFF_DO, sP = base + C::OFF_P, sDS = base + C::OFF_DS;
+    uint32_t it = 0, unit_it = 0, dq_issued = 0;
+    auto kdesc = [](uint32_t a) { return sdesc_sw128(a, 16, 1024); };
+    // S (or dP) = X Y^T over d = 256: X a [128][256] tile, Y a [64][256] tile
+    auto mma_qk = [&](uint32_t d_t, uint32_t x, uint32_t y) {
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            const uint32_t xa = x + (kk >> 2) * C::Q_BLK + (kk & 3) * 32u;
+            const uint32_t ya = y + (kk >> 2) * C::KV_BLK + (kk & 3) * 32u;
+            mma_ss(tmem + d_t, kdesc(xa), kdesc(ya), C::IDESC_S, kk > 0);
+        }
+    };
+    // acc^T[half] (+)= X^T Z: X a [128 query][256] tile read MN-major (head-dim half
+    // `hf`), Z a [128 query][64 key] tile read MN-major
+    auto mma_t = [&](uint32_t d_t, uint32_t x, uint32_t z, bool acc) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + d_t + hf * 64, sdesc_sw128(x + 2 * hf * C::Q_BLK + kk * 2048u, C::Q_BLK, 1024),
+                       sdesc_sw128(z + kk * 2048u, C::Q_BLK, 1024), C::IDESC_T, (acc || kk > 0) ? 1u : 0u);
+    };
+    // dQ half `dh` = dS K[:, 128 dh .. 128 dh + 127]
+    auto mma_dq = [&](int dh) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + C::T_DQ, kdesc(sDS + kk * 32u),
+                   sdesc_sw128(sK + 2 * dh * C::KV_BLK + kk * 2048u, C::KV_BLK, 1024), C::IDESC_Q, kk > 0);
+    };
+    auto wait_dq_free = [&]() -> bool {
+        if (dq_issued == 0) return true;
+        return wait_fast(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_B256_DQ_EMPTY);
+    };
+    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+        const BwdUnit u = bwd256_decode(p, ui);
+        if (u.T == 0) continue;
+        if (!wait_fast(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_B256_KV_FULL)) return;
+        tc_fence_after();
+        if (!wait_fast(bar(C::B_Q_FULL), it & 1u, ctl, W_B256_Q_FULL)) return;
+        tc_fence_after();
+        mma_qk(C::T_S, sQ, sK);
+        mma_commit(bar(C::B_S_FULL));
+        if (!wait_fast(bar(C::B_DO_FULL), it & 1u, ctl, W_B256_DO_FULL)) return;
+        tc_fence_after();
+        mma_qk(C::T_DP, sDO, sV);
+        mma_commit(bar(C::B_DP_FULL));
+        for (int s = 0; s < u.T; ++s, ++it) {
+            if (!wait_fast(bar(C::B_P_FULL), it & 1u, ctl, W_B256_P_FULL)) return;
+            tc_fence_after();
+            mma_t(C::T_DV, sDO, sP, s > 0);
+            mma_commit(bar(C::B_P_EMPTY));
+            mma_commit(bar(C::B_DO_EMPTY));
+            if (!wait_fast(bar(C::B_DS_FULL), it & 1u, ctl, W_B256_DS_FULL)) return;
+            tc_fence_after();
+            mma_t(C::T_DK, sQ, sDS, s > 0);
+            mma_commit(bar(C::B_Q_EMPTY));
+            if (!wait_dq_free()) return;
+            tc_fence_after();
+            mma_dq(0);
+            mma_commit(bar(C::B_DQ_FULL));
+            ++dq_issued;
+            if (s + 1 < u.T) {
+                if (!wait_fast(bar(C::B_Q_FULL), (it + 1) & 1u, ctl, W_B256_Q_FULL)) return;
+                tc_fence_after();
+                mma_qk(C::T_S, sQ, sK);
+                mma_commit(bar(C::B_S_FULL));
+                if (!wait_fast(bar(C::B_DO_FULL), (it + 1) & 1u, ctl, W_B256_DO_FULL)) return;
+                tc_fence_after();
+                mma_qk(C::T_DP, sDO, sV);
+                mma_commit(bar(C::B_DP_FULL));
+            }
+            if (!wait_dq_free()) return;
+            tc_fence_after();
+            mma_dq(1);
+            mma_commit(bar(C::B_DQ_FULL));
+            ++dq_issued;
+            mma_commit(bar(C::B_DS_EMPTY));
+        }
+        mma_commit(bar(C::B_KV_EMPTY));
+        mma_commit(bar(C::B_DKV_FINAL));
+        ++unit_it;
+    }
+}
+
+// ---- TMA producer --------------------------------------------------------------------
+template <bool BF16>
+struct Bwd256Load {
+    using C = Bwd256Cfg<BF16>;
+    const CUtensorMap *tmQ, *tmK, *tmV, *tmDO;  // K, V maps have 64-row boxes
+    uint32_t base, bars;
+    CtaCtl* ctl;
+    int kv_round = -1, q_round = -1, do_round = -1;
+
+    __device__ uint32_t bar(int i) const { return bars + 8u * i; }
+    __device__ void run(const BwdParams& p)
+    {
+        uint32_t it = 0, unit_it = 0;
+        for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+            const BwdUnit u = bwd256_decode(p, ui);
+            if (u.T == 0) continue;
+            if (!wait_bar(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_B256_KV_EMPTY)) return;
+            mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::KV_BYTES);
+            for (int blk = 0; blk < 4; ++blk) {
+                tma_load_4d(base + C::OFF_K + blk * C::KV_BLK, tmK, bar(C::B_KV_FULL), blk * 64, u.hkv, u.n * 64, u.b);
+                tma_load_4d(base + C::OFF_V + blk * C::KV_BLK, tmV, bar(C::B_KV_FULL), blk * 64, u.hkv, u.n * 64, u.b);
+            }
+            kv_round = static_cast<int>(unit_it);
+            ++unit_it;
+            for (int s = 0; s < u.T; ++s, ++it) {
+                int h, m;
+                bwd_step(p, u, s, h, m);
+                const uint32_t ph = (it & 1u) ^ 1u;
+                if (!wait_bar(bar(C::B_Q_EMPTY), ph, ctl, W_B256_Q_EMPTY)) return;
+                mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_BYTES + C::ROWS_BYTES);
+                for (int blk = 0; blk < 4; ++blk)
+                    tma_load_4d(base + C::OFF_Q + blk * C::Q_BLK, tmQ, bar(C::B_Q_FULL), blk * 64, h, m * 128, u.b);
+                {
+                    const size_t rb = (static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + static_cast<size_t>(m) * 128;
+                    bulk_load(base + C::OFF_ROWS, p.L2 + rb, 512, bar(C::B_Q_FULL));
+                    bulk_load(base + C::OFF_ROWS + 512, p.Dv + rb, 512, bar(C::B_Q_FULL));
+                }
+                q_round = static_cast<int>(it);
+                if (!wait_bar(bar(C::B_DO_EMPTY), ph, ctl, W_B256_DO_EMPTY)) return;
+                mbar_arrive_expect_tx(bar(C::B_DO_FULL), C::Q_BYTES);
+                for (int blk = 0; blk < 4; ++blk)
+                    tma_load_4d(base + C::OFF_DO + blk * C::Q_BLK, tmDO, bar(C::B_DO_FULL), blk * 64, h, m * 128, u.b);
+                do_round = static_cast<int>(it);
+            }
+        }
+    }
+    __device__ void drain()
+    {
+        if (kv_round >= 0) drain_wait(bar(C::B_KV_FULL), static_cast<uint32_t>(kv_round) & 1u, W_B256_DRAIN);
+        if (q_round >= 0) drain_wait(bar(C::B_Q_FULL), static_cast<uint32_t>(q_round) & 1u, W_B256_DRAIN);
+        if (do_round >= 0) drain_wait(bar(C::B_DO_FULL), static_cast<uint32_t>(do_round) & 1u, W_B256_DRAIN);
+    }
+};
+
+template <bool BF16>
+__global__ void __launch_bounds__(Bwd256Cfg<BF16>::THREADS, 1)
+    fa_bwd_dkdv256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                          const BwdParams p)
+{
+    using C = Bwd256Cfg<BF16>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base = smem_u32(smem_raw);
+    if (base & 1023u) {  // swizzled TMA tiles and MMA descriptors need 1024-byte alignment
+        if (threadIdx.x == 0 &&
+            atomicCAS(&g_status[0], 0u, static_cast<uint32_t>(FA_ERR_UNSUPPORTED)) == 0u)
+            g_status[1] = W_B256_SMEM_ALIGN;
+        return;
+    }
+    const uint32_t bars = base + C::OFF_BAR;
+    CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem_raw + C::OFF_CTL);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        auto bar = [&](int i) { return bars + 8u * i; };
+        for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), 1);
+        mbar_init(bar(C::B_P_FULL), 4);
+        mbar_init(bar(C::B_DS_FULL), 4);
+        mbar_init(bar(C::B_DQ_EMPTY), 4);
+        ctl->abort = 0u;
+        fence_mbar_init();
+    }
+    if (warp == C::MMA_WARP) {
+        tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+        tmem_relinquish();
+    }
+    if (warp == C::LOAD_WARP && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmDO);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp < 4) {
+        bwd256_compute<BF16>(p, tmem, base, bars, ctl, warp);
+    } else if (warp < 8) {
+        bwd256_dq_reduce<BF16>(p, tmem, bars, ctl, warp - 4);
+    } else if (warp == C::MMA_WARP) {
+        if (lane == 0) {
+            bwd256_mma<BF16>(p, tmem, base, bars, ctl);
+            mma_commit(bars + 8u * C::B_DRAIN);
+            drain_wait(bars + 8u * C::B_DRAIN, 0u, W_B256_DRAIN);
+        }
+        __syncwarp();
+    } else if (warp == C::LOAD_WARP) {
+        if (lane == 0) {
+            Bwd256Load<BF16> ld{&tmQ, &tmK, &tmV, &tmDO, base, bars, ctl};
+            ld.run(p);
+            ld.drain();
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == C::MMA_WARP) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace fa

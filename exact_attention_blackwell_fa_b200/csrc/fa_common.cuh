@@ -66,13 +66,74 @@ __device__ __noinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32_t 
     return true;
 }
 
-// Warp-wide wait: lane 0 polls, the result is broadcast (the shuffle also syncs the warp).
+// Single-thread wait with an inline first probe (the common case: already complete).
+__device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, CtaCtl* ctl,
+                                          uint32_t where)
+{
+    return mbar_try_wait(bar, parity) || wait_bar(bar, parity, ctl, where);
+}
+
+// Warp-wide wait: lane 0 polls (its successful wait is the acquire), the result is
+// broadcast, and a warp barrier -- which orders memory among the lanes, unlike the
+// shuffle -- makes everything lane 0 acquired visible to the other lanes' later loads.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, CtaCtl* ctl,
                                           uint32_t where)
 {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, ctl, where) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_fast(bar, parity, ctl, where) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// ---------------------------------------------------------------------------------
+// Packed fp32 pairs (sm_100 f32x2 arithmetic on the FMA pipe: two lanes of work per
+// instruction).  A pair lives in one 64-bit register, `lo` in the low half.
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2unpack(uint64_t v)
+{
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// exp2_fma on a pair with packed arithmetic; same steps and constants as exp2_fma.
+__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& e0, float& e1)
+{
+    const uint64_t x = f2pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+    const uint64_t t = fadd2(x, f2pack(12582912.0f, 12582912.0f));
+    const uint64_t n = fadd2(t, f2pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = ffma2(n, f2pack(-1.0f, -1.0f), x);  // x - n, exact
+    uint64_t p = ffma2(f2pack(FA_EXP2_C3, FA_EXP2_C3), f, f2pack(FA_EXP2_C2, FA_EXP2_C2));
+    p = ffma2(p, f, f2pack(FA_EXP2_C1, FA_EXP2_C1));
+    p = ffma2(p, f, f2pack(FA_EXP2_C0, FA_EXP2_C0));
+    const float2 pf = f2unpack(p), tf = f2unpack(t);
+    e0 = __int_as_float(__float_as_int(pf.x) + (__float_as_int(tf.x) << 23));
+    e1 = __int_as_float(__float_as_int(pf.y) + (__float_as_int(tf.y) << 23));
 }
 
 // ---------------------------------------------------------------------------------
@@ -87,6 +148,20 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
     } else {
         __half2 v = __floats2half2_rn(lo, hi);
         return *reinterpret_cast<uint32_t*>(&v);
+    }
+}
+
+// Packing of P (values in [0, 2^8]) for the P V product.  bf16: round to nearest with
+// ties away from zero done with integer adds and a byte permute, which keeps the
+// conversion off the special-function pipe that the SFU exponentials already load;
+// fp16: the hardware conversion (round to nearest even).
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2_p(float lo, float hi)
+{
+    if constexpr (BF16) {
+        return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+    } else {
+        return pack2<false>(lo, hi);
     }
 }
 

@@ -11,16 +11,19 @@
 //     (batch, query head, block of query rows); units are grouped by heads so that the
 //     CTAs running at the same time share K/V through L2, and for the causal mask the
 //     longest units (last query blocks) go first;
-//   * one TMA warp stages Q once per unit and streams K and V through a 5-deep ring
+//   * one TMA warp stages Q once per unit and streams K and V through a 4-deep ring
 //     of 32-KB shared-memory chunks (128 rows x 128 head-dim columns, 128-byte
 //     swizzle) guarded by full/empty mbarriers;
 //   * one thread issues tcgen05.mma: S = Q K^T into TMEM, then O += P V with P read
 //     back from TMEM (P overwrites the first half of its own S buffer as 16-bit
 //     pairs);
-//   * softmax warpgroups (thread = query row) load S from TMEM, apply the scale and
-//     mask, keep the running row max / sum, rescale O in TMEM only when the row max
-//     grew by more than kRescaleTau (log2 units), compute P with exp2 split between
-//     the SFU and an FMA-pipe cubic, and finally normalise O and write O and LSE.
+//   * two softmax warpgroups per Q tile, each owning 64 of the 128 key columns of
+//     every query row (thread = query row): they load their half of S from TMEM,
+//     apply the scale and mask, swap half-row maxima through shared memory, keep the
+//     running row max / half-row sum, rescale their half of O in TMEM only when the
+//     row max grew by more than kRescaleTau (log2 units), compute P with exp2 split
+//     between the SFU and an FMA-pipe cubic, and finally normalise and write their
+//     half of O (the halves' row sums are combined once per unit);
 //
 // head_dim 128: two Q tiles (256 query rows) per unit, TMEM = S0 | S1 | O0 | O1; the
 // tensor core alternates between the two tiles so that one tile's softmax overlaps
@@ -53,7 +56,8 @@ struct FwdParams {
 // wait-site codes reported through the device status word
 enum : uint32_t {
     W_FWD_Q_FULL = 0x101, W_FWD_Q_EMPTY, W_FWD_RING_FULL, W_FWD_RING_EMPTY, W_FWD_S_FULL,
-    W_FWD_P_FULL, W_FWD_O_DONE, W_FWD_O_FINAL, W_FWD_DRAIN
+    W_FWD_P_FULL, W_FWD_O_DONE, W_FWD_O_FINAL, W_FWD_DRAIN, W_FWD_XMAX, W_FWD_XSUM,
+    W_FWD_SMEM_ALIGN
 };
 
 template <int D, bool BF16>
@@ -62,20 +66,25 @@ struct FwdCfg {
     static constexpr int NQ = D == 128 ? 2 : 1;  // 128-row Q tiles per work unit
     static constexpr int NS = D == 128 ? 1 : 2;  // S buffers per Q tile
     static constexpr int KCH = D / 128;          // 32-KB chunks per K (or V) tile
-    static constexpr int NSTAGE = 5;             // ring depth, in chunks
+    static constexpr int NSTAGE = 4;             // ring depth, in chunks
     static constexpr int BM = 128;               // query rows per Q tile
     static constexpr int BN = 128;               // keys per KV tile
+    static constexpr int HALF = 64;              // key columns per softmax warpgroup
     static constexpr int UNIT_ROWS = NQ * BM;
     static constexpr uint32_t CHUNK = 32768;
     static constexpr uint32_t QTILE = BM * D * 2;
     static constexpr uint32_t Q_BYTES = NQ * QTILE;
-    static constexpr int THREADS = (NQ + 1) * 128;
-    static constexpr int CTRL_WARP = NQ * 4;  // MMA warp; the TMA warp follows it
+    static constexpr int SOFTMAX_WARPS = NQ * 8;     // two warpgroups per Q tile
+    static constexpr int CTRL_WARP = SOFTMAX_WARPS;  // MMA warp; the TMA warp follows it
+    static constexpr int THREADS = (SOFTMAX_WARPS + 2) * 32;
 
-    // shared memory map (offsets from a 1024-aligned base)
+    // shared memory map (offsets from the 1024-aligned dynamic shared memory base)
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_RING = Q_BYTES;
-    static constexpr uint32_t OFF_BAR = OFF_RING + NSTAGE * CHUNK;
+    // half-row maxima, [Q tile][step parity][half][row], then half-row sums [Q tile][half][row]
+    static constexpr uint32_t OFF_XMAX = OFF_RING + NSTAGE * CHUNK;
+    static constexpr uint32_t OFF_XSUM = OFF_XMAX + NQ * 2 * 2 * BM * 4;
+    static constexpr uint32_t OFF_BAR = OFF_XSUM + NQ * 2 * BM * 4;
     // barrier indices
     static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1;
     static constexpr int B_FULL = 2;
@@ -84,14 +93,21 @@ struct FwdCfg {
     static constexpr int B_P_FULL = B_S_FULL + NQ * NS;
     static constexpr int B_O_DONE = B_P_FULL + NQ * NS;
     static constexpr int B_O_FINAL = B_O_DONE + NQ;
-    static constexpr int B_DRAIN = B_O_FINAL + NQ;
+    static constexpr int B_XMAX = B_O_FINAL + NQ;  // [Q tile][step parity]
+    static constexpr int B_XSUM = B_XMAX + 2 * NQ;
+    static constexpr int B_DRAIN = B_XSUM + NQ;
     static constexpr int NBAR = B_DRAIN + 1;
     static constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
-    static constexpr uint32_t SMEM_BYTES = OFF_CTL + sizeof(CtaCtl) + 1024;
+    // no alignment slack: the kernel checks that the base is 1024-byte aligned
+    static constexpr uint32_t SMEM_BYTES = OFF_CTL + sizeof(CtaCtl);
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
     // TMEM columns
     __device__ static constexpr uint32_t col_S(int q, int sb) { return NQ == 2 ? q * 128 : sb * 128; }
     __device__ static constexpr uint32_t col_O(int q) { return 256 + q * 128; }
+    // P for key columns 64h .. 64h+63 is written by softmax half h over the first 32
+    // columns of its own (already consumed) half of the S buffer
+    __device__ static constexpr uint32_t col_P(int half) { return half * 64; }
 
     static constexpr uint32_t IDESC_S = idesc_f16(BF16, 128, 128, false, false);
     static constexpr uint32_t IDESC_PV = idesc_f16(BF16, 128, 128, false, true);
@@ -127,19 +143,23 @@ __device__ __forceinline__ int fwd_kv_tiles(const FwdParams& p, int m0)
 }
 
 // ---------------------------------------------------------------------------------
-// Softmax / epilogue warpgroup (one per Q tile).
+// Softmax / epilogue warpgroups: two per Q tile, `half` owns key columns 64h..64h+63.
 // ---------------------------------------------------------------------------------
 template <int D, bool BF16>
-__device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int q,
-                            int wq)
+__device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, uint8_t* smem,
+                            CtaCtl* ctl, int q, int half, int wq)
 {
     using C = FwdCfg<D, BF16>;
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    constexpr int OCOLS = D / 2;  // O columns this warpgroup rescales and stores
     const int lane = threadIdx.x & 31;
     const int r_in_tile = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tO = tmem + lane_off + C::col_O(q);
+    const uint32_t tO = tmem + lane_off + C::col_O(q) + half * OCOLS;
+    float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX) + q * (2 * 2 * C::BM);
+    float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM) + q * (2 * C::BM);
     auto bar = [&](int i) { return bars + 8u * i; };
+    const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
     uint32_t s_it = 0, pv_it = 0, tile_it = 0;
 
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
@@ -149,14 +169,15 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, Ct
         const int q0 = m0 + q * C::BM;  // first query row of this Q tile
         const int row = q0 + r_in_tile;
         const bool row_ok = row < p.Sq;
-        T* orow = reinterpret_cast<T*>(p.o) + ((static_cast<size_t>(b) * p.Sq + row) * p.Hq + h) * D;
+        T* orow = reinterpret_cast<T*>(p.o) + ((static_cast<size_t>(b) * p.Sq + row) * p.Hq + h) * D +
+                  half * OCOLS;
         float* lrow = p.lse + (static_cast<size_t>(b) * p.Hq + h) * p.Sq + row;
         if (n == 0) {  // causal with Sq > Sk: no key is visible to any row of the unit
             if (row_ok) {
-                uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
-                *lrow = -INFINITY;
+                for (int c = 0; c < OCOLS / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
+                if (half == 0) *lrow = -INFINITY;
             }
             continue;
         }
@@ -165,30 +186,45 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, Ct
         const int lim = p.causal ? min(p.Sk, row + p.Sk - p.Sq + 1) : p.Sk;
         const int lim0 = p.causal ? min(p.Sk, q0 + p.Sk - p.Sq + 1) : p.Sk;
 
-        float m_ref = -INFINITY;  // running reference max (log2 units)
-        float l = 0.0f;           // running row sum against m_ref
+        float m_ref = -INFINITY;  // running reference max (log2 units), same in both halves
+        float l = 0.0f;           // running sum of this half's columns against m_ref
         for (int j = 0; j < n; ++j) {
             const int sb = s_it % C::NS;
             if (!warp_wait(bar(C::B_S_FULL + q * C::NS + sb), (s_it / C::NS) & 1u, ctl, W_FWD_S_FULL))
                 return;
             tc_fence_after();
-            const uint32_t tS = tmem + lane_off + C::col_S(q, sb);
-            uint32_t sr[128];
-            tmem_ld128_wait(tS, sr);
-            const bool masked = (j + 1) * C::BN > lim0;
+            const uint32_t tS = tmem + lane_off + C::col_S(q, sb) + half * C::HALF;
+            uint32_t r0[32], r1[32];
+            tmem_ld32_nowait(tS, r0);
+            tmem_ld32_nowait(tS + 32, r1);
+            tmem_wait_ld_dep(r0);
+            tmem_wait_ld_dep(r1);
+            const int c0 = j * C::BN + half * C::HALF;  // key index of column 0 of this half
+            const bool masked = c0 + C::HALF > lim0;
             if (masked) {
-                const int cut = lim - j * C::BN;
+                const int cut = lim - c0;
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c >= cut) sr[c] = __float_as_uint(-INFINITY);
+                for (int c = 0; c < 32; ++c) {
+                    if (c >= cut) r0[c] = __float_as_uint(-INFINITY);
+                    if (c + 32 >= cut) r1[c] = __float_as_uint(-INFINITY);
+                }
             }
-            float mx[8];
+            float mx[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sr[i]);
+            for (int i = 0; i < 4; ++i) mx[i] = fmaxf(__uint_as_float(r0[i]), __uint_as_float(r1[i]));
 #pragma unroll
-            for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
-            const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            for (int c = 4; c < 32; c += 4)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    mx[i] = fmax3(mx[i], __uint_as_float(r0[c + i]), __uint_as_float(r1[c + i]));
+            const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            // swap half-row maxima with the other warpgroup of this Q tile
+            const int par = s_it & 1;
+            xmax[(par * 2 + half) * C::BM + r_in_tile] = hmax;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_XMAX + q * 2 + par));
+            if (!warp_wait(bar(C::B_XMAX + q * 2 + par), (s_it >> 1) & 1u, ctl, W_FWD_XMAX)) return;
+            const float rmax = fmaxf(hmax, xmax[(par * 2 + (half ^ 1)) * C::BM + r_in_tile]);
             const float m_tile = rmax * p.sl2;  // scale > 0, so max commutes with it
             const float m_new = fmaxf(m_ref, m_tile);
             const bool resc = (m_ref != -INFINITY) && (m_new - m_ref > kRescaleTau);
@@ -203,7 +239,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, Ct
                 }
                 const float alpha = resc ? ex2_sfu(m_ref - m_new) : 1.0f;
 #pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
+                for (int cc = 0; cc < OCOLS / 32; ++cc) {
                     uint32_t r[32];
                     tmem_ld32_wait(tO + cc * 32, r);
 #pragma unroll
@@ -217,30 +253,44 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, Ct
                 }
             }
             const float negm = (m_ref == -INFINITY) ? 0.0f : -m_ref;
-            float sum[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint64_t negm2 = f2pack(negm, negm);
+            uint64_t sum2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
+            const uint32_t tP = tmem + lane_off + C::col_S(q, sb) + C::col_P(half);
+            // the S values are loaded again, 32 columns at a time, to keep the register
+            // footprint small (the second load is in flight while the first is used)
+            tmem_ld32_nowait(tS, r0);
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < 2; ++cc) {
+                uint32_t (&r)[32] = cc == 0 ? r0 : r1;
+                tmem_wait_ld_dep(r);
+                if (cc == 0) tmem_ld32_nowait(tS + 32, r1);
+                if (masked) {
+                    const int cut = lim - c0 - cc * 32;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (c >= cut) r[c] = __float_as_uint(-INFINITY);
+                }
                 uint32_t pk[16];
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
-                    const float x0 = fmaf(__uint_as_float(sr[cc * 32 + k]), p.sl2, negm);
-                    const float x1 = fmaf(__uint_as_float(sr[cc * 32 + k + 1]), p.sl2, negm);
+                    const float2 x = f2unpack(ffma2(f2pack(__uint_as_float(r[k]), __uint_as_float(r[k + 1])),
+                                                    sl2x2, negm2));
                     float e0, e1;
-                    // 1 of every 4 exponentials on the FMA pipe (unmasked tiles only:
-                    // the SFU maps -inf to exactly 0)
+                    // exponentials of alternate pairs on the FMA pipe (packed cubic), the
+                    // rest on the SFU; masked tiles use the SFU only (it maps -inf to 0)
                     if (!masked && (k & 2)) {
-                        e0 = exp2_fma(x0);
-                        e1 = ex2_sfu(x1);
+                        exp2_fma_x2(x.x, x.y, e0, e1);
                     } else {
-                        e0 = ex2_sfu(x0);
-                        e1 = ex2_sfu(x1);
+                        e0 = ex2_sfu(x.x);
+                        e1 = ex2_sfu(x.y);
                     }
-                    sum[(k >> 1) & 3] += e0 + e1;
-                    pk[k >> 1] = pack2<BF16>(e0, e1);
+                    sum2[(k >> 1) & 1] = fadd2(sum2[(k >> 1) & 1], f2pack(e0, e1));
+                    pk[k >> 1] = pack2_p<BF16>(e0, e1);
                 }
-                tmem_st16(tS + cc * 16, pk);
+                tmem_st16(tP + cc * 16, pk);
             }
-            l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+            const float2 s0 = f2unpack(sum2[0]), s1 = f2unpack(sum2[1]);
+            l += (s0.x + s0.y) + (s1.x + s1.y);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -248,13 +298,19 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, Ct
             ++s_it;
             ++pv_it;
         }
-        // epilogue: wait for the unit's last P V, normalise, store O and LSE
+        // epilogue: combine the halves' row sums, wait for the unit's last P V,
+        // normalise and store this half of O (and LSE, from half 0)
+        xsum[half * C::BM + r_in_tile] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_XSUM + q));
+        if (!warp_wait(bar(C::B_XSUM + q), tile_it & 1u, ctl, W_FWD_XSUM)) return;
+        const float l_all = l + xsum[(half ^ 1) * C::BM + r_in_tile];
         if (!warp_wait(bar(C::B_O_FINAL + q), tile_it & 1u, ctl, W_FWD_O_FINAL)) return;
         ++tile_it;
         tc_fence_after();
-        const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
+        const float inv = (l_all > 0.0f) ? 1.0f / l_all : 0.0f;
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
+        for (int cc = 0; cc < OCOLS / 32; ++cc) {
             uint32_t r[32];
             tmem_ld32_wait(tO + cc * 32, r);
             uint32_t pk[16];
@@ -269,7 +325,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, Ct
                 dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
             }
         }
-        if (row_ok) *lrow = (l > 0.0f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (row_ok && half == 0)
+            *lrow = (l_all > 0.0f) ? (m_ref + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
         tc_fence_before();
     }
 }
@@ -309,7 +366,8 @@ struct FwdMma {
     {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t a = tmem + C::col_S(q, sb) + kk * 8;
+            // k-steps 0-3 read P of key columns 0-63 (half 0), 4-7 of 64-127 (half 1)
+            const uint32_t a = tmem + C::col_S(q, sb) + C::col_P(kk >> 2) + (kk & 3) * 8;
 #pragma unroll
             for (int c = 0; c < C::KCH; ++c) {
                 const uint32_t bv = slot(sV + c) + kk * 2048u;
@@ -524,13 +582,17 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
 {
     using C = FwdCfg<D, BF16>;
     extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* base_ptr = smem_raw + (base - raw);
+    const uint32_t base = smem_u32(smem_raw);
+    if (base & 1023u) {  // swizzled TMA tiles and MMA descriptors need 1024-byte alignment
+        if (threadIdx.x == 0 &&
+            atomicCAS(&g_status[0], 0u, static_cast<uint32_t>(FA_ERR_UNSUPPORTED)) == 0u)
+            g_status[1] = W_FWD_SMEM_ALIGN;
+        return;
+    }
     const uint32_t sQ = base + C::OFF_Q;
     const uint32_t sRing = base + C::OFF_RING;
     const uint32_t bars = base + C::OFF_BAR;
-    CtaCtl* ctl = reinterpret_cast<CtaCtl*>(base_ptr + C::OFF_CTL);
+    CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem_raw + C::OFF_CTL);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -544,11 +606,14 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
         }
         for (int i = 0; i < C::NQ * C::NS; ++i) {
             mbar_init(bar(C::B_S_FULL + i), 1);
-            mbar_init(bar(C::B_P_FULL + i), 4);  // one arrive per softmax warp
+            mbar_init(bar(C::B_P_FULL + i), 8);  // one arrive per softmax warp of the tile
         }
         for (int q = 0; q < C::NQ; ++q) {
             mbar_init(bar(C::B_O_DONE + q), 1);
             mbar_init(bar(C::B_O_FINAL + q), 1);
+            mbar_init(bar(C::B_XMAX + 2 * q), 8);
+            mbar_init(bar(C::B_XMAX + 2 * q + 1), 8);
+            mbar_init(bar(C::B_XSUM + q), 8);
         }
         mbar_init(bar(C::B_DRAIN), 1);
         ctl->abort = 0u;
@@ -568,8 +633,8 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
 
-    if (warp < C::NQ * 4) {
-        fwd_softmax<D, BF16>(p, tmem, bars, ctl, warp >> 2, warp & 3);
+    if (warp < C::SOFTMAX_WARPS) {
+        fwd_softmax<D, BF16>(p, tmem, bars, smem_raw, ctl, warp >> 3, (warp >> 2) & 1, warp & 3);
     } else if (warp == C::CTRL_WARP) {
         if (lane == 0) {
             FwdMma<D, BF16> mma{tmem, sQ, sRing, bars, ctl};

@@ -62,6 +62,10 @@ SMALL = [
     (1, 200, 333, 2, 1, 128),
     (1, 1, 1, 1, 1, 128),
     (1, 130, 1, 2, 2, 128),
+    (1, 256, 256, 2, 2, 256),
+    (2, 300, 200, 4, 2, 256),     # head_dim 256: 64-key units, ragged tails, GQA
+    (1, 200, 333, 2, 1, 256),
+    (1, 1, 1, 1, 1, 256),
 ]
 
 
@@ -71,9 +75,10 @@ def test_bwd_small_bf16(oracle_mod, shape, causal):
     check_full(oracle_mod, Shape(*shape), causal)
 
 
-def test_bwd_fp16(oracle_mod):
-    check_full(oracle_mod, Shape(1, 320, 320, 2, 2, 128), True, dtype=torch.float16)
-    check_full(oracle_mod, Shape(1, 320, 320, 2, 2, 128), False, dtype=torch.float16)
+@pytest.mark.parametrize("d", [128, 256])
+def test_bwd_fp16(oracle_mod, d):
+    check_full(oracle_mod, Shape(1, 320, 320, 2, 2, d), True, dtype=torch.float16)
+    check_full(oracle_mod, Shape(1, 320, 320, 2, 2, d), False, dtype=torch.float16)
 
 
 def test_bwd_causal_rows_without_keys(oracle_mod):
@@ -85,7 +90,16 @@ def test_bwd_causal_rows_without_keys(oracle_mod):
     assert_grads(dq, dk, dv, rq, rk, rv)
 
 
-def test_bwd_many_units(oracle_mod):
+@pytest.mark.parametrize("d", [128, 256])
+def test_bwd_many_units(oracle_mod, d):
     """More key blocks than SMs, GQA group of 4, causal: persistent CTAs walk several
     units; dQ partials from many CTAs meet in the fp32 accumulator."""
-    check_full(oracle_mod, Shape(2, 1024, 1024, 8, 2, 128), True)
+    check_full(oracle_mod, Shape(2, 1024, 1024, 8, 2, d), True)
+
+
+def test_bwd_causal_rows_without_keys_d256(oracle_mod):
+    shape = Shape(1, 500, 100, 2, 1, 256)
+    (q, k, v, do), dq, dk, dv = run_bwd(shape, True)
+    rq, rk, rv, _ = oracle_mod.bwd(q, k, v, do, causal=True)
+    assert torch.all(dq[:, :400] == 0)
+    assert_grads(dq, dk, dv, rq, rk, rv)
