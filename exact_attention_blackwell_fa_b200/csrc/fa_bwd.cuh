@@ -402,72 +402,79 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32
 {
     using C = BwdCfg<BF16>;
     auto bar = [&](int i) { return bars + 8u * i; };
-    const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sDS = base + C::OFF_DS;
     uint32_t it = 0, unit_it = 0, dq_issued = 0;
-    auto kdesc = [](uint32_t a) { return sdesc_sw128(a, 16, 1024); };
-    auto mdesc = [](uint32_t a) { return sdesc_sw128(a, 16384, 1024); };
+    // Descriptors are built once; each MMA adds a constant byte offset / 16 to the
+    // start-address field (addresses stay below 256 KB, so it cannot carry).
+    const uint64_t kK = sdesc_sw128(base + C::OFF_K, 16, 1024);      // K, K-major
+    const uint64_t kV = sdesc_sw128(base + C::OFF_V, 16, 1024);      // V, K-major
+    const uint64_t mK = sdesc_sw128(base + C::OFF_K, 16384, 1024);   // K, MN-major
+    const uint64_t kQ = sdesc_sw128(base + C::OFF_Q, 16, 1024);      // Q stage 0, K-major
+    const uint64_t mQ = sdesc_sw128(base + C::OFF_Q, 16384, 1024);   // Q stage 0, MN-major
+    const uint64_t kDO = sdesc_sw128(base + C::OFF_DO, 16, 1024);
+    const uint64_t mDO = sdesc_sw128(base + C::OFF_DO, 16384, 1024);
+    const uint64_t kDS = sdesc_sw128(base + C::OFF_DS, 16, 1024);    // dS^T, K-major
+    const uint64_t mDS = sdesc_sw128(base + C::OFF_DS, 16384, 1024); // dS^T, MN-major
+    constexpr uint64_t STAGE = C::TILE >> 4;
     // S^T (or dP^T) = A B^T over d, both K-major tiles
-    auto mma_kk = [&](uint32_t d_t, uint32_t a, uint32_t b) {
+    auto mma_kk = [&](uint32_t d_t, uint64_t a, uint64_t b) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-            mma_ss(tmem + d_t, kdesc(a + off), kdesc(b + off), C::IDESC_KK, kk > 0);
+            const uint32_t off = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
+            mma_ss(tmem + d_t, a + off, b + off, C::IDESC_KK, kk > 0);
         }
     };
     auto wait_dq_free = [&]() -> bool {
         if (dq_issued == 0) return true;
-        return wait_bar(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_BWD_DQ_EMPTY);
+        return wait_fast(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_BWD_DQ_EMPTY);
     };
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
         const BwdUnit u = bwd_decode(p, ui);
         if (u.T == 0) continue;
-        if (!wait_bar(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_BWD_KV_FULL)) return;
+        if (!wait_fast(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_BWD_KV_FULL)) return;
         tc_fence_after();
         {
             const int st = it & 1;
-            if (!wait_bar(bar(C::B_Q_FULL + st), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
+            if (!wait_fast(bar(C::B_Q_FULL + st), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
             tc_fence_after();
-            mma_kk(C::T_S, sK, base + C::OFF_Q + st * C::TILE);
+            mma_kk(C::T_S, kK, kQ + st * STAGE);
             mma_commit(bar(C::B_S_FULL));
             if (!wait_dq_free()) return;
-            if (!wait_bar(bar(C::B_DO_FULL + st), (it >> 1) & 1u, ctl, W_BWD_DO_FULL)) return;
+            if (!wait_fast(bar(C::B_DO_FULL + st), (it >> 1) & 1u, ctl, W_BWD_DO_FULL)) return;
             tc_fence_after();
-            mma_kk(C::T_DP, sV, base + C::OFF_DO + st * C::TILE);
+            mma_kk(C::T_DP, kV, kDO + st * STAGE);
             mma_commit(bar(C::B_DP_FULL));
         }
         for (int s = 0; s < u.T; ++s, ++it) {
             const int st = it & 1;
-            const uint32_t sQ = base + C::OFF_Q + st * C::TILE;
-            const uint32_t sDO = base + C::OFF_DO + st * C::TILE;
+            const uint64_t mQs = mQ + st * STAGE, mDOs = mDO + st * STAGE;
             // dV += P^T dO
-            if (!wait_bar(bar(C::B_P_FULL), it & 1u, ctl, W_BWD_P_FULL)) return;
+            if (!wait_fast(bar(C::B_P_FULL), it & 1u, ctl, W_BWD_P_FULL)) return;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8, mdesc(sDO + kk * 2048u), C::IDESC_KM,
+                mma_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8, mDOs + kk * 128u, C::IDESC_KM,
                        (s > 0 || kk > 0) ? 1u : 0u);
             mma_commit(bar(C::B_DO_EMPTY + st));
             // next S^T as soon as P^T has been consumed (in-order tensor pipe)
             const int nst = (it + 1) & 1;
             if (s + 1 < u.T) {
-                if (!wait_bar(bar(C::B_Q_FULL + nst), ((it + 1) >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
+                if (!wait_fast(bar(C::B_Q_FULL + nst), ((it + 1) >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
                 tc_fence_after();
-                mma_kk(C::T_S, sK, base + C::OFF_Q + nst * C::TILE);
+                mma_kk(C::T_S, kK, kQ + nst * STAGE);
                 mma_commit(bar(C::B_S_FULL));
             }
             // dK += dS^T Q ; dQ_part = dS K
-            if (!wait_bar(bar(C::B_DS_FULL), it & 1u, ctl, W_BWD_DS_FULL)) return;
+            if (!wait_fast(bar(C::B_DS_FULL), it & 1u, ctl, W_BWD_DS_FULL)) return;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t a = sDS + (kk >> 2) * 16384u + (kk & 3) * 32u;
-                mma_ss(tmem + C::T_DK, kdesc(a), mdesc(sQ + kk * 2048u), C::IDESC_KM,
+                const uint32_t off = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
+                mma_ss(tmem + C::T_DK, kDS + off, mQs + kk * 128u, C::IDESC_KM,
                        (s > 0 || kk > 0) ? 1u : 0u);
             }
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + C::T_DP, mdesc(sDS + kk * 2048u), mdesc(sK + kk * 2048u), C::IDESC_MM,
-                       kk > 0 ? 1u : 0u);
+                mma_ss(tmem + C::T_DP, mDS + kk * 128u, mK + kk * 128u, C::IDESC_MM, kk > 0 ? 1u : 0u);
             mma_commit(bar(C::B_DQ_FULL));
             ++dq_issued;
             mma_commit(bar(C::B_Q_EMPTY + st));
@@ -475,9 +482,9 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32
             // next dP^T once the dQ readers have drained TMEM
             if (s + 1 < u.T) {
                 if (!wait_dq_free()) return;
-                if (!wait_bar(bar(C::B_DO_FULL + nst), ((it + 1) >> 1) & 1u, ctl, W_BWD_DO_FULL)) return;
+                if (!wait_fast(bar(C::B_DO_FULL + nst), ((it + 1) >> 1) & 1u, ctl, W_BWD_DO_FULL)) return;
                 tc_fence_after();
-                mma_kk(C::T_DP, sV, base + C::OFF_DO + nst * C::TILE);
+                mma_kk(C::T_DP, kV, kDO + nst * STAGE);
                 mma_commit(bar(C::B_DP_FULL));
             }
         }

@@ -264,32 +264,37 @@ __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uin
     const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQ = base + C::OFF_Q,
                    sDO = base + C::OFF_DO, sP = base + C::OFF_P, sDS = base + C::OFF_DS;
     uint32_t it = 0, unit_it = 0, dq_issued = 0;
-    auto kdesc = [](uint32_t a) { return sdesc_sw128(a, 16, 1024); };
+    // descriptors built once; each MMA adds a constant byte offset / 16 (see fa_bwd.cuh)
+    const uint64_t kQ = sdesc_sw128(sQ, 16, 1024), kDO = sdesc_sw128(sDO, 16, 1024);
+    const uint64_t kK = sdesc_sw128(sK, 16, 1024), kV = sdesc_sw128(sV, 16, 1024);
+    const uint64_t mQ = sdesc_sw128(sQ, C::Q_BLK, 1024), mDO = sdesc_sw128(sDO, C::Q_BLK, 1024);
+    const uint64_t mP = sdesc_sw128(sP, C::Q_BLK, 1024), mDS = sdesc_sw128(sDS, C::Q_BLK, 1024);
+    const uint64_t kDS = sdesc_sw128(sDS, 16, 1024), mK = sdesc_sw128(sK, C::KV_BLK, 1024);
     // S (or dP) = X Y^T over d = 256: X a [128][256] tile, Y a [64][256] tile
-    auto mma_qk = [&](uint32_t d_t, uint32_t x, uint32_t y) {
+    auto mma_qk = [&](uint32_t d_t, uint64_t x, uint64_t y) {
 #pragma unroll
         for (int kk = 0; kk < 16; ++kk) {
-            const uint32_t xa = x + (kk >> 2) * C::Q_BLK + (kk & 3) * 32u;
-            const uint32_t ya = y + (kk >> 2) * C::KV_BLK + (kk & 3) * 32u;
-            mma_ss(tmem + d_t, kdesc(xa), kdesc(ya), C::IDESC_S, kk > 0);
+            const uint32_t xo = ((kk >> 2) * C::Q_BLK + (kk & 3) * 32u) >> 4;
+            const uint32_t yo = ((kk >> 2) * C::KV_BLK + (kk & 3) * 32u) >> 4;
+            mma_ss(tmem + d_t, x + xo, y + yo, C::IDESC_S, kk > 0);
         }
     };
     // acc^T[half] (+)= X^T Z: X a [128 query][256] tile read MN-major (head-dim half
     // `hf`), Z a [128 query][64 key] tile read MN-major
-    auto mma_t = [&](uint32_t d_t, uint32_t x, uint32_t z, bool acc) {
+    auto mma_t = [&](uint32_t d_t, uint64_t x, uint64_t z, bool acc) {
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + d_t + hf * 64, sdesc_sw128(x + 2 * hf * C::Q_BLK + kk * 2048u, C::Q_BLK, 1024),
-                       sdesc_sw128(z + kk * 2048u, C::Q_BLK, 1024), C::IDESC_T, (acc || kk > 0) ? 1u : 0u);
+                mma_ss(tmem + d_t + hf * 64, x + ((2 * hf * C::Q_BLK + kk * 2048u) >> 4), z + kk * 128u,
+                       C::IDESC_T, (acc || kk > 0) ? 1u : 0u);
     };
     // dQ half `dh` = dS K[:, 128 dh .. 128 dh + 127]
     auto mma_dq = [&](int dh) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + C::T_DQ, kdesc(sDS + kk * 32u),
-                   sdesc_sw128(sK + 2 * dh * C::KV_BLK + kk * 2048u, C::KV_BLK, 1024), C::IDESC_Q, kk > 0);
+            mma_ss(tmem + C::T_DQ, kDS + kk * 2u, mK + ((2 * dh * C::KV_BLK + kk * 2048u) >> 4), C::IDESC_Q,
+                   kk > 0);
     };
     auto wait_dq_free = [&]() -> bool {
         if (dq_issued == 0) return true;
@@ -302,21 +307,21 @@ __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uin
         tc_fence_after();
         if (!wait_fast(bar(C::B_Q_FULL), it & 1u, ctl, W_B256_Q_FULL)) return;
         tc_fence_after();
-        mma_qk(C::T_S, sQ, sK);
+        mma_qk(C::T_S, kQ, kK);
         mma_commit(bar(C::B_S_FULL));
         if (!wait_fast(bar(C::B_DO_FULL), it & 1u, ctl, W_B256_DO_FULL)) return;
         tc_fence_after();
-        mma_qk(C::T_DP, sDO, sV);
+        mma_qk(C::T_DP, kDO, kV);
         mma_commit(bar(C::B_DP_FULL));
         for (int s = 0; s < u.T; ++s, ++it) {
             if (!wait_fast(bar(C::B_P_FULL), it & 1u, ctl, W_B256_P_FULL)) return;
             tc_fence_after();
-            mma_t(C::T_DV, sDO, sP, s > 0);
+            mma_t(C::T_DV, mDO, mP, s > 0);
             mma_commit(bar(C::B_P_EMPTY));
             mma_commit(bar(C::B_DO_EMPTY));
             if (!wait_fast(bar(C::B_DS_FULL), it & 1u, ctl, W_B256_DS_FULL)) return;
             tc_fence_after();
-            mma_t(C::T_DK, sQ, sDS, s > 0);
+            mma_t(C::T_DK, mQ, mDS, s > 0);
             mma_commit(bar(C::B_Q_EMPTY));
             if (!wait_dq_free()) return;
             tc_fence_after();
@@ -326,11 +331,11 @@ __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uin
             if (s + 1 < u.T) {
                 if (!wait_fast(bar(C::B_Q_FULL), (it + 1) & 1u, ctl, W_B256_Q_FULL)) return;
                 tc_fence_after();
-                mma_qk(C::T_S, sQ, sK);
+                mma_qk(C::T_S, kQ, kK);
                 mma_commit(bar(C::B_S_FULL));
                 if (!wait_fast(bar(C::B_DO_FULL), (it + 1) & 1u, ctl, W_B256_DO_FULL)) return;
                 tc_fence_after();
-                mma_qk(C::T_DP, sDO, sV);
+                mma_qk(C::T_DP, kDO, kV);
                 mma_commit(bar(C::B_DP_FULL));
             }
             if (!wait_dq_free()) return;

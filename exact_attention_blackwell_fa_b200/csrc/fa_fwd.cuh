@@ -159,7 +159,6 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, ui
     float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX) + q * (2 * 2 * C::BM);
     float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM) + q * (2 * C::BM);
     auto bar = [&](int i) { return bars + 8u * i; };
-    const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
     uint32_t s_it = 0, pv_it = 0, tile_it = 0;
 
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
@@ -218,80 +217,114 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, ui
                 for (int i = 0; i < 4; ++i)
                     mx[i] = fmax3(mx[i], __uint_as_float(r0[c + i]), __uint_as_float(r1[c + i]));
             const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            // swap half-row maxima with the other warpgroup of this Q tile
+            // publish this half-row maximum to the other warpgroup of the Q tile
             const int par = s_it & 1;
             xmax[(par * 2 + half) * C::BM + r_in_tile] = hmax;
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_XMAX + q * 2 + par));
-            if (!warp_wait(bar(C::B_XMAX + q * 2 + par), (s_it >> 1) & 1u, ctl, W_FWD_XMAX)) return;
-            const float rmax = fmaxf(hmax, xmax[(par * 2 + (half ^ 1)) * C::BM + r_in_tile]);
-            const float m_tile = rmax * p.sl2;  // scale > 0, so max commutes with it
-            const float m_new = fmaxf(m_ref, m_tile);
-            const bool resc = (m_ref != -INFINITY) && (m_new - m_ref > kRescaleTau);
-            if (m_ref == -INFINITY) m_ref = m_new;
-            if (__any_sync(0xffffffffu, resc)) {
-                // O must hold every earlier P V product before it is scaled: with one S
-                // buffer that is implied by S_full (the MMA issued S after the previous
-                // P V); with two, wait for the previous P V explicitly.
-                if (C::NS == 2) {
-                    if (!warp_wait(bar(C::B_O_DONE + q), (pv_it - 1u) & 1u, ctl, W_FWD_O_DONE)) return;
-                    tc_fence_after();
-                }
-                const float alpha = resc ? ex2_sfu(m_ref - m_new) : 1.0f;
-#pragma unroll 1
-                for (int cc = 0; cc < OCOLS / 32; ++cc) {
-                    uint32_t r[32];
-                    tmem_ld32_wait(tO + cc * 32, r);
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-                    tmem_st32(tO + cc * 32, r);
-                }
-                tmem_wait_st();
-                if (resc) {
-                    l *= alpha;
-                    m_ref = m_new;
-                }
-            }
-            const float negm = (m_ref == -INFINITY) ? 0.0f : -m_ref;
-            const uint64_t negm2 = f2pack(negm, negm);
-            uint64_t sum2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
-            const uint32_t tP = tmem + lane_off + C::col_S(q, sb) + C::col_P(half);
-            // the S values are loaded again, 32 columns at a time, to keep the register
-            // footprint small (the second load is in flight while the first is used)
-            tmem_ld32_nowait(tS, r0);
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                uint32_t (&r)[32] = cc == 0 ? r0 : r1;
-                tmem_wait_ld_dep(r);
-                if (cc == 0) tmem_ld32_nowait(tS + 32, r1);
-                if (masked) {
-                    const int cut = lim - c0 - cc * 32;
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (c >= cut) r[c] = __float_as_uint(-INFINITY);
-                }
-                uint32_t pk[16];
-#pragma unroll
-                for (int k = 0; k < 32; k += 2) {
-                    const float2 x = f2unpack(ffma2(f2pack(__uint_as_float(r[k]), __uint_as_float(r[k + 1])),
-                                                    sl2x2, negm2));
-                    float e0, e1;
-                    // exponentials of alternate pairs on the FMA pipe (packed cubic), the
-                    // rest on the SFU; masked tiles use the SFU only (it maps -inf to 0)
-                    if (!masked && (k & 2)) {
-                        exp2_fma_x2(x.x, x.y, e0, e1);
-                    } else {
-                        e0 = ex2_sfu(x.x);
-                        e1 = ex2_sfu(x.y);
+
+            // Reference update for the whole row: both halves see the same two maxima and
+            // reach the same decision.
+            auto update_reference = [&](float partner) -> bool {
+                const float m_tile = fmaxf(hmax, partner) * p.sl2;  // scale > 0
+                const float m_new = fmaxf(m_ref, m_tile);
+                const bool resc = (m_ref != -INFINITY) && (m_new - m_ref > kRescaleTau);
+                if (m_ref == -INFINITY) m_ref = m_new;
+                if (__any_sync(0xffffffffu, resc)) {
+                    // O must hold every earlier P V product before it is scaled: with one
+                    // S buffer that is implied by S_full (the MMA issued S after the
+                    // previous P V); with two, wait for the previous P V explicitly.
+                    if (C::NS == 2) {
+                        if (!warp_wait(bar(C::B_O_DONE + q), (pv_it - 1u) & 1u, ctl, W_FWD_O_DONE))
+                            return false;
+                        tc_fence_after();
                     }
-                    sum2[(k >> 1) & 1] = fadd2(sum2[(k >> 1) & 1], f2pack(e0, e1));
-                    pk[k >> 1] = pack2_p<BF16>(e0, e1);
+                    const float alpha = resc ? ex2_sfu(m_ref - m_new) : 1.0f;
+#pragma unroll 1
+                    for (int cc = 0; cc < OCOLS / 32; ++cc) {
+                        uint32_t r[32];
+                        tmem_ld32_wait(tO + cc * 32, r);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+                        tmem_st32(tO + cc * 32, r);
+                    }
+                    tmem_wait_st();
+                    if (resc) {
+                        l *= alpha;
+                        m_ref = m_new;
+                    }
                 }
-                tmem_st16(tP + cc * 16, pk);
+                return true;
+            };
+            const uint32_t tP = tmem + lane_off + C::col_S(q, sb) + C::col_P(half);
+            // P = 2^(S scale log2e - m_ref) for this half, into registers: the S values are
+            // loaded again, 32 columns at a time (the second load in flight while the first
+            // is used), which keeps the register footprint small.  S stays intact in TMEM
+            // until store_p, so the pass can be redone.
+            uint32_t pk[32];
+            auto exp_pass = [&]() -> float {
+                const float negm = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                tmem_ld32_nowait(tS, r0);
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t (&r)[32] = cc == 0 ? r0 : r1;
+                    tmem_wait_ld_dep(r);
+                    if (cc == 0) tmem_ld32_nowait(tS + 32, r1);
+                    if (masked) {
+                        const int cut = lim - c0 - cc * 32;
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (c >= cut) r[c] = __float_as_uint(-INFINITY);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 32; k += 2) {
+                        const float x0 = fmaf(__uint_as_float(r[k]), p.sl2, negm);
+                        const float x1 = fmaf(__uint_as_float(r[k + 1]), p.sl2, negm);
+                        float e0, e1;
+                        // one pair in four on the FMA pipe (packed cubic), the rest on the
+                        // SFU; masked tiles use the SFU only (it maps -inf to exactly 0)
+                        if (!masked && (k & 6) == 6) {
+                            exp2_fma_x2(x0, x1, e0, e1);
+                        } else {
+                            e0 = ex2_sfu(x0);
+                            e1 = ex2_sfu(x1);
+                        }
+                        acc[(k >> 1) & 3] += e0 + e1;
+                        pk[cc * 16 + (k >> 1)] = pack2_p<BF16>(e0, e1);
+                    }
+                }
+                return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            };
+            // P overwrites the first 32 columns of this half's (consumed) S columns
+            auto store_p = [&]() {
+                const uint32_t tP = tmem + lane_off + C::col_S(q, sb) + C::col_P(half);
+                tmem_st16(tP, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+                tmem_st16(tP + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+                tmem_wait_st();
+            };
+            const float m_loc = hmax * p.sl2;
+            // With an established reference and this half's maximum within kRescaleTau of it
+            // (the common case after the first tile), P is computed before the other half's
+            // maximum is known; if that maximum then forces a new reference, the pass is
+            // redone.  Otherwise the maxima are swapped first.
+            const bool speculate =
+                !__any_sync(0xffffffffu, m_ref == -INFINITY || m_loc - m_ref > kRescaleTau);
+            float tile_sum;
+            if (speculate) {
+                tile_sum = exp_pass();
+                if (!warp_wait(bar(C::B_XMAX + q * 2 + par), (s_it >> 1) & 1u, ctl, W_FWD_XMAX)) return;
+                const float partner = xmax[(par * 2 + (half ^ 1)) * C::BM + r_in_tile];
+                const float m_before = m_ref;
+                if (!update_reference(partner)) return;
+                if (__any_sync(0xffffffffu, m_ref != m_before)) tile_sum = exp_pass();
+            } else {
+                if (!warp_wait(bar(C::B_XMAX + q * 2 + par), (s_it >> 1) & 1u, ctl, W_FWD_XMAX)) return;
+                if (!update_reference(xmax[(par * 2 + (half ^ 1)) * C::BM + r_in_tile])) return;
+                tile_sum = exp_pass();
             }
-            const float2 s0 = f2unpack(sum2[0]), s1 = f2unpack(sum2[1]);
-            l += (s0.x + s0.y) + (s1.x + s1.y);
-            tmem_wait_st();
+            store_p();
+            l += tile_sum;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q * C::NS + sb));
@@ -349,31 +382,53 @@ struct FwdMma {
     }
     __device__ void release(uint32_t s) { mma_commit(bar(C::B_EMPTY + s % C::NSTAGE)); }
 
+    // Descriptors are built once; every MMA then only adds a constant byte offset / 16
+    // to the 14-bit start-address field (it cannot carry: addresses stay below 256 KB).
+    // This keeps the single issuing thread's instruction count per MMA small -- it
+    // shares its scheduler with busy softmax warps.
+    uint64_t qdesc0 = 0, kdesc0 = 0, vdesc0 = 0;
+    __device__ void init_descs()
+    {
+        qdesc0 = sdesc_sw128(sQ, 16, 1024);
+        kdesc0 = sdesc_sw128(sRing, 16, 1024);
+        vdesc0 = sdesc_sw128(sRing, 16384, 1024);
+    }
+    __device__ uint64_t slot_off(uint32_t s) const
+    {
+        return static_cast<uint64_t>((s % C::NSTAGE) * (C::CHUNK >> 4));
+    }
+
     // S(q, sb) = Q_q K^T, K tile in ring chunks sK .. sK + KCH - 1
     __device__ void issue_S(int q, int sb, uint32_t sK)
     {
         const uint32_t d = tmem + C::col_S(q, sb);
+        const uint64_t qd = qdesc0 + static_cast<uint64_t>(q * (C::QTILE >> 4));
+        uint64_t kd[C::KCH];
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c) kd[c] = kdesc0 + slot_off(sK + c);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t a = sQ + q * C::QTILE + (kk >> 2) * 16384u + (kk & 3) * 32u;
-            const uint32_t bk = slot(sK + (kk >> 3)) + ((kk & 7) >> 2) * 16384u + (kk & 3) * 32u;
-            mma_ss(d, sdesc_sw128(a, 16, 1024), sdesc_sw128(bk, 16, 1024), C::IDESC_S, kk > 0);
+            const uint32_t aoff = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
+            const uint32_t boff = (((kk & 7) >> 2) * 16384u + (kk & 3) * 32u) >> 4;
+            mma_ss(d, qd + aoff, kd[kk >> 3] + boff, C::IDESC_S, kk > 0);
         }
     }
     // O_q (+)= P(q, sb) V, V tile in ring chunks sV .. sV + KCH - 1 (chunk c = O columns
     // c*128 .. c*128+127)
     __device__ void issue_PV(int q, int sb, uint32_t sV, bool acc)
     {
+        uint64_t vd[C::KCH];
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c) vd[c] = vdesc0 + slot_off(sV + c);
+        const uint32_t tP = tmem + C::col_S(q, sb);
+        const uint32_t tO = tmem + C::col_O(q);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             // k-steps 0-3 read P of key columns 0-63 (half 0), 4-7 of 64-127 (half 1)
-            const uint32_t a = tmem + C::col_S(q, sb) + C::col_P(kk >> 2) + (kk & 3) * 8;
+            const uint32_t a = tP + C::col_P(kk >> 2) + (kk & 3) * 8;
 #pragma unroll
-            for (int c = 0; c < C::KCH; ++c) {
-                const uint32_t bv = slot(sV + c) + kk * 2048u;
-                mma_ts(tmem + C::col_O(q) + c * 128, a, sdesc_sw128(bv, 16384, 1024), C::IDESC_PV,
-                       (acc || kk > 0) ? 1u : 0u);
-            }
+            for (int c = 0; c < C::KCH; ++c)
+                mma_ts(tO + c * 128, a, vd[c] + (kk * 2048u >> 4), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
     }
     __device__ bool wait_chunks(uint32_t s0)
@@ -638,6 +693,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
     } else if (warp == C::CTRL_WARP) {
         if (lane == 0) {
             FwdMma<D, BF16> mma{tmem, sQ, sRing, bars, ctl};
+            mma.init_descs();
             mma.run(p);
             // all MMAs issued by this thread must finish before TMEM is released
             mma_commit(bars + 8u * C::B_DRAIN);

@@ -119,3 +119,44 @@ def test_fwd_many_units_persistent(oracle_mod):
     assert_o_close(got, o_ref, torch.bfloat16)
     lerr = (lse[rows[:, 0], rows[:, 1], rows[:, 2]].double() - lse_ref).abs().max().item()
     assert lerr <= LSE_MAX
+
+
+def _growing_keys(shape, upper_half_only, dtype=torch.bfloat16):
+    """Keys whose norm grows along the sequence, so the running row maximum keeps
+    jumping by more than the rescale threshold from one KV tile to the next.  With
+    upper_half_only, only keys in columns 64..127 of each 128-key tile grow, so one
+    half-row's maximum jumps while the other's does not."""
+    q, k, v = make_inputs(shape, seed=7, dtype=dtype)
+    Sk = shape.Sk
+    gain = torch.linspace(0.2, 12.0, Sk)
+    if upper_half_only:
+        gain = torch.where((torch.arange(Sk) % 128) >= 64, gain, torch.full_like(gain, 0.2))
+    k = (k.float() * gain.view(1, Sk, 1, 1)).to(dtype)
+    return q, k, v
+
+
+@pytest.mark.parametrize("upper_half_only", [False, True])
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_rescale_paths(oracle_mod, upper_half_only, d, causal):
+    """Exercise the thresholded O rescale, including a reference jump seen by only one
+    of the two half-row warpgroups.  These keys are far from N(0, 1) and make most rows
+    attend to one or two keys, so the bound is the one the arithmetic fixes rather than
+    the N(0, 1) tolerance: P is rounded to bf16 (unit roundoff u = 2^-8) before P V,
+    giving |dO_i| <= u * sum_j P_ij |v_j| <= u * max |v| per element (plus the output
+    rounding) and about u * mean |v| on average."""
+    import exact_attention_blackwell_fa_b200 as fa
+
+    shape = Shape(1, 256, 1024, 2, 2, d)
+    q, k, v = _growing_keys(shape, upper_half_only)
+    o, lse = fa.fa_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle_mod.fwd(q, k, v, causal=causal)
+    err = (o.cpu().double() - o_ref).abs()
+    assert torch.isfinite(err).all()
+    bound = p_rounding_bound(v, torch.bfloat16) + half_ulp(o_ref, torch.bfloat16)
+    assert (err - bound).max().item() <= 0.0, f"O max abs err {err.max().item()}"
+    assert err.mean().item() <= 2.0 ** -8 * v.double().abs().mean().item(), err.mean().item()
+    fin = torch.isfinite(lse_ref)
+    assert (lse.cpu().double()[fin] - lse_ref[fin]).abs().max().item() <= LSE_MAX * max(
+        1.0, lse_ref[fin].abs().max().item() / 100.0)
