@@ -97,6 +97,18 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(value, device):
+    """Maximum of a per-rank time over all ranks (the step time of the slowest
+    replica); the value itself when not running distributed."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def oracle_cpu_baseline(budget_s=15.0):
     """Time the fp64 oracle on a bounded sample of the workload: full-length query rows
     of one head through the forward (O, LSE) and the backward dQ path.  Returns the
@@ -252,11 +264,7 @@ def main():
     end.record(stream)
     barrier()
     clocks = sampler.stop()
-    total_ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(end), dev)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) if do_bwd else 0.0
     ms_per_step = total_ms / K
@@ -296,11 +304,7 @@ def main():
                 hdv.copy_(dv, non_blocking=True)
         e1.record(stream)
         barrier()
-        e2e_ms = e0.elapsed_time(e1) / E
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / E, dev)
         e2e = {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 

@@ -1,0 +1,46 @@
+"""Bounded waits: a kernel that never receives one of its tiles reports
+FA_ERR_DEVICE_TIMEOUT instead of hanging, and the context stays usable.
+
+The failure is made on the host: fa_debug_inject(1) makes the next forward launch
+withhold its first K tile copy, so the MMA issuer's wait for it runs out (about one
+second); every other wait then sees the CTA's abort flag, in-flight copies and MMAs
+are drained, TMEM is freed and the kernel returns.  No trap, fault or unbounded
+spin is involved.
+"""
+import time
+
+import pytest
+import torch
+
+from exact_attention_blackwell_fa_b200.inputs import Shape, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+FA_ERR_DEVICE_TIMEOUT = 4
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_withheld_tile_reports_timeout_then_recovers(oracle_mod, d):
+    import exact_attention_blackwell_fa_b200 as fa
+
+    shape = Shape(1, 256, 256, 2, 2, d)
+    q, k, v = make_inputs(shape, seed=3)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    fa.fa_clear_device_status()
+    torch.cuda.synchronize()
+    fa.fa_debug_inject(1)
+    t0 = time.time()
+    fa.fa_fwd(qc, kc, vc)
+    torch.cuda.synchronize()
+    elapsed = time.time() - t0
+    code, detail = fa.fa_last_device_status()
+    assert code == FA_ERR_DEVICE_TIMEOUT, (code, hex(detail))
+    assert 0x100 <= detail < 0x200, hex(detail)  # a forward wait site gave up
+    assert elapsed < 30.0
+    # the context is still usable and the next launch is correct
+    fa.fa_clear_device_status()
+    o, lse = fa.fa_fwd(qc, kc, vc)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status()[0] == 0
+    o_ref, _ = oracle_mod.fwd(q, k, v)
+    assert (o.cpu().double() - o_ref).abs().max().item() <= 1.2e-2
