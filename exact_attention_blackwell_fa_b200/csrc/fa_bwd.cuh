@@ -18,8 +18,9 @@
 //        compute warpgroup (thread = key row): P^T -> TMEM as 16-bit pairs,
 //                                               dS^T -> shared memory (swizzled)
 //        dV += P^T dO   (A from TMEM)           dK += dS^T Q   (A K-major)
-//        dQ_part = dS K (A = the same dS^T tile read MN-major) -> TMEM -> fp32
-//        vector reductions into the dQ accumulator by a second warpgroup;
+//        dQ^T = K^T dS^T (both read MN-major; head dims land on the TMEM lanes)
+//        -> fp32 reductions into the dQ accumulator by a second warpgroup, one
+//        128-byte accumulator segment per warp instruction;
 //   3. convert: dQ = scale * accumulator, in the input dtype and layout.
 #pragma once
 
@@ -266,13 +267,10 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
                         const float la = e == 0 ? l4.x : l4.z, lb = e == 0 ? l4.y : l4.w;
                         const float2 x = f2unpack(ffma2(f2pack(__uint_as_float(r[k]), __uint_as_float(r[k + 1])),
                                                         sl2x2, f2pack(-la, -lb)));
-                        float e0, e1;
-                        if (!masked && (k & 2)) {
-                            exp2_fma_x2(x.x, x.y, e0, e1);
-                        } else {
-                            e0 = ex2_sfu(x.x);
-                            e1 = ex2_sfu(x.y);
-                        }
+                        // all on the SFU: 128x128 exponentials per step are ~1k SFU cycles,
+                        // well under the step's tensor time, and this warpgroup has no
+                        // spare warps to hide the longer FMA-pipe sequence
+                        float e0 = ex2_sfu(x.x), e1 = ex2_sfu(x.y);
                         if (masked) {
                             const int c = cc * 32 + k;
                             if (c < jlim) e0 = 0.0f;
@@ -369,7 +367,7 @@ __device__ void bwd_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, 
 {
     using C = BwdCfg<BF16>;
     const int lane = threadIdx.x & 31;
-    const int t = wq * 32 + lane;  // query row within the block
+    const int t = wq * 32 + lane;  // head dim (= TMEM lane of dQ^T)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     auto bar = [&](int i) { return bars + 8u * i; };
     uint32_t it = 0;
@@ -380,17 +378,17 @@ __device__ void bwd_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, 
             bwd_step(p, u, s, h, m);
             if (!warp_wait(bar(C::B_DQ_FULL), it & 1u, ctl, W_BWD_DQ_FULL)) return;
             tc_fence_after();
-            uint32_t r[128];
+            uint32_t r[128];  // r[i] = dQ^T[dim t][query i] of this block
             tmem_ld128_wait(tmem + lane_off + C::T_DP, r);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
-            float* dst = p.dqacc + ((static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + m * 128 + t) * C::D;
+            // lanes hold consecutive dims, so each warp-wide reduction covers 128
+            // contiguous bytes of one accumulator row
+            float* dst = p.dqacc + ((static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + m * 128) * C::D + t;
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * c),
-                             "f"(__uint_as_float(r[4 * c])), "f"(__uint_as_float(r[4 * c + 1])),
-                             "f"(__uint_as_float(r[4 * c + 2])), "f"(__uint_as_float(r[4 * c + 3]))
+            for (int i = 0; i < 128; ++i)
+                asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst + i * C::D), "f"(__uint_as_float(r[i]))
                              : "memory");
         }
     }
@@ -463,7 +461,7 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32
                 mma_kk(C::T_S, kK, kQ + nst * STAGE);
                 mma_commit(bar(C::B_S_FULL));
             }
-            // dK += dS^T Q ; dQ_part = dS K
+            // dK += dS^T Q ; dQ^T = K^T dS^T
             if (!wait_fast(bar(C::B_DS_FULL), it & 1u, ctl, W_BWD_DS_FULL)) return;
             tc_fence_after();
 #pragma unroll
@@ -472,9 +470,10 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32
                 mma_ss(tmem + C::T_DK, kDS + off, mQs + kk * 128u, C::IDESC_KM,
                        (s > 0 || kk > 0) ? 1u : 0u);
             }
+            // dQ^T = K^T dS^T: head dims on the TMEM lanes (both operands MN-major)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + C::T_DP, mDS + kk * 128u, mK + kk * 128u, C::IDESC_MM, kk > 0 ? 1u : 0u);
+                mma_ss(tmem + C::T_DP, mK + kk * 128u, mDS + kk * 128u, C::IDESC_MM, kk > 0 ? 1u : 0u);
             mma_commit(bar(C::B_DQ_FULL));
             ++dq_issued;
             mma_commit(bar(C::B_Q_EMPTY + st));
