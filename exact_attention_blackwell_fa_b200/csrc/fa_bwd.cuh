@@ -15,8 +15,8 @@
 //      (batch, KV head); it loops over every query head of the KV group and every
 //      block of 128 query rows.  Per step, all in TMEM:
 //        S^T = K Q^T,  dP^T = V dO^T            (tcgen05, A and B K-major)
-//        compute warpgroup (thread = key row): P^T -> TMEM as 16-bit pairs,
-//                                               dS^T -> shared memory (swizzled)
+//        two compute warpgroups (thread = key row; one warpgroup per half of the
+//        128 query columns): P^T -> TMEM as 16-bit pairs, dS^T -> shared memory
 //        dV += P^T dO   (A from TMEM)           dK += dS^T Q   (A K-major)
 //        dQ^T = K^T dS^T (both read MN-major; head dims land on the TMEM lanes)
 //        -> fp32 reductions into the dQ accumulator by a second warpgroup, one
@@ -153,8 +153,9 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p)
 template <bool BF16>
 struct BwdCfg {
     static constexpr int D = 128;
-    static constexpr int THREADS = 384;
-    static constexpr int MMA_WARP = 8, LOAD_WARP = 9;
+    // warps 0-7: compute (two warpgroups, one per 64-query half), 8-11: dQ, 12: MMA, 13: TMA
+    static constexpr int THREADS = 448;
+    static constexpr int DQ_WARP = 8, MMA_WARP = 12, LOAD_WARP = 13;
     static constexpr uint32_t TILE = 32768;  // 128 rows x 128 columns x 2 bytes
     // per query block: LSE*log2(e) and D for its 128 rows, staged with the Q tile
     static constexpr uint32_t ROWS_BYTES = 1024;
@@ -218,14 +219,17 @@ __device__ __forceinline__ void bwd_step(const BwdParams& p, const BwdUnit& u, i
 // ---- compute warpgroup: P^T and dS^T, then the dK / dV epilogue --------------------
 template <bool BF16>
 __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uint32_t sRows,
-                            uint32_t bars, CtaCtl* ctl, int wq)
+                            uint32_t bars, CtaCtl* ctl, int wq, int half)
 {
     using C = BwdCfg<BF16>;
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
     const int lane = threadIdx.x & 31;
     const int t = wq * 32 + lane;  // key row within the block (= TMEM lane)
+    const int q0 = half * 64;      // this warpgroup's query columns: q0 .. q0 + 63
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::T_S, tDP = tmem + lane_off + C::T_DP;
+    // S^T / dP^T columns of this half; P^T goes to the first 32 columns of the half
+    // (16-bit pairs), below the S^T columns still to be read
+    const uint32_t tS = tmem + lane_off + C::T_S + q0, tDP = tmem + lane_off + C::T_DP + q0;
     auto bar = [&](int i) { return bars + 8u * i; };
     const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
     uint32_t it = 0, unit_it = 0;
@@ -238,7 +242,7 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
             const uint32_t rows = sRows + (it & 1) * C::ROWS_BYTES;  // L2[128] then D[128]
             // key j is visible to query i iff j <= i + (Sk - Sq)
             const bool masked = p.causal && (u.n * 128 + 127 > m * 128 + p.Sk - p.Sq);
-            const int jlim = j - (p.Sk - p.Sq) - m * 128;  // visible iff column c >= jlim
+            const int jlim = j - (p.Sk - p.Sq) - m * 128 - q0;  // visible iff column c >= jlim
             // the Q-tile barrier also covers the staged row terms
             if (!warp_wait(bar(C::B_Q_FULL + (it & 1)), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
             if (!warp_wait(bar(C::B_S_FULL), it & 1u, ctl, W_BWD_S_FULL)) return;
@@ -246,21 +250,21 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
             // P^T = 2^(S^T scale log2e - LSE log2e), 32 query columns at a time.  The
             // 16-bit P^T words stay in registers for dS: the MMA issues the next S^T into
             // these TMEM columns as soon as dV has consumed them.
-            uint32_t ppk[64];
+            uint32_t ppk[32];
             uint32_t rbuf[2][32];
             tmem_ld32_nowait(tS, rbuf[0]);
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < 2; ++cc) {
                 uint32_t (&r)[32] = rbuf[cc & 1];
                 tmem_wait_ld_dep(r);
-                if (cc + 1 < 4) tmem_ld32_nowait(tS + (cc + 1) * 32, rbuf[(cc + 1) & 1]);
+                if (cc + 1 < 2) tmem_ld32_nowait(tS + (cc + 1) * 32, rbuf[(cc + 1) & 1]);
                 uint32_t (&pk)[16] = *reinterpret_cast<uint32_t(*)[16]>(&ppk[cc * 16]);
 #pragma unroll
                 for (int k4 = 0; k4 < 8; ++k4) {
                     float4 l4;
                     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                                  : "=f"(l4.x), "=f"(l4.y), "=f"(l4.z), "=f"(l4.w)
-                                 : "r"(rows + (cc * 32 + k4 * 4) * 4u));
+                                 : "r"(rows + (q0 + cc * 32 + k4 * 4) * 4u));
 #pragma unroll
                     for (int e = 0; e < 4; e += 2) {
                         const int k = k4 * 4 + e;
@@ -292,19 +296,19 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
             tc_fence_after();
             tmem_ld32_nowait(tDP, rbuf[0]);
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < 2; ++cc) {
                 uint32_t (&r)[32] = rbuf[cc & 1];
                 tmem_wait_ld_dep(r);
-                if (cc + 1 < 4) tmem_ld32_nowait(tDP + (cc + 1) * 32, rbuf[(cc + 1) & 1]);
+                if (cc + 1 < 2) tmem_ld32_nowait(tDP + (cc + 1) * 32, rbuf[(cc + 1) & 1]);
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {  // 8 query columns -> one 16-byte chunk
                     float4 da, db;
                     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                                  : "=f"(da.x), "=f"(da.y), "=f"(da.z), "=f"(da.w)
-                                 : "r"(rows + 512u + (cc * 32 + g * 8) * 4u));
+                                 : "r"(rows + 512u + (q0 + cc * 32 + g * 8) * 4u));
                     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                                  : "=f"(db.x), "=f"(db.y), "=f"(db.z), "=f"(db.w)
-                                 : "r"(rows + 512u + (cc * 32 + g * 8 + 4) * 4u));
+                                 : "r"(rows + 512u + (q0 + cc * 32 + g * 8 + 4) * 4u));
                     const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
                     uint32_t q4[4];
 #pragma unroll
@@ -314,7 +318,7 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
                         q4[w] = pack2<BF16>(pp.x * (__uint_as_float(r[k]) - dv[w * 2]),
                                             pp.y * (__uint_as_float(r[k + 1]) - dv[w * 2 + 1]));
                     }
-                    const int col8 = cc * 4 + g;  // 8-column group 0..15
+                    const int col8 = half * 8 + cc * 4 + g;  // 8-column group 0..15
                     const uint32_t addr = sDS + (col8 >> 3) * 16384u + t * 128u +
                                           ((static_cast<uint32_t>(col8 & 7) ^ (t & 7)) << 4);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(q4[0]),
@@ -341,7 +345,7 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
             T* dst = which == 0 ? dvrow : dkrow;
             const uint32_t col = which == 0 ? C::T_DV : C::T_DK;
 #pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
                 uint32_t r[32];
                 tmem_ld32_wait(tmem + lane_off + col + cc * 32, r);
                 uint32_t pk[16];
@@ -378,18 +382,34 @@ __device__ void bwd_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, 
             bwd_step(p, u, s, h, m);
             if (!warp_wait(bar(C::B_DQ_FULL), it & 1u, ctl, W_BWD_DQ_FULL)) return;
             tc_fence_after();
-            uint32_t r[128];  // r[i] = dQ^T[dim t][query i] of this block
-            tmem_ld128_wait(tmem + lane_off + C::T_DP, r);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
             // lanes hold consecutive dims, so each warp-wide reduction covers 128
-            // contiguous bytes of one accumulator row
+            // contiguous bytes of one accumulator row.  Two 64-query halves (the
+            // register budget of this 14-warp block); TMEM is released after the
+            // second half has been read, the first half's reductions already issued.
             float* dst = p.dqacc + ((static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + m * 128) * C::D + t;
 #pragma unroll
-            for (int i = 0; i < 128; ++i)
-                asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst + i * C::D), "f"(__uint_as_float(r[i]))
-                             : "memory");
+            for (int hq = 0; hq < 2; ++hq) {
+                uint32_t r0[32], r1[32];  // dQ^T[dim t][query 64 hq + i]
+                tmem_ld32_nowait(tmem + lane_off + C::T_DP + hq * 64, r0);
+                tmem_ld32_nowait(tmem + lane_off + C::T_DP + hq * 64 + 32, r1);
+                tmem_wait_ld_dep(r0);
+                tmem_wait_ld_dep(r1);
+                if (hq == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
+                }
+                float* d0 = dst + hq * 64 * C::D;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(d0 + i * C::D), "f"(__uint_as_float(r0[i]))
+                                 : "memory");
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(d0 + (32 + i) * C::D),
+                                 "f"(__uint_as_float(r1[i]))
+                                 : "memory");
+            }
         }
     }
 }
@@ -448,10 +468,11 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32
             // dV += P^T dO
             if (!wait_fast(bar(C::B_P_FULL), it & 1u, ctl, W_BWD_P_FULL)) return;
             tc_fence_after();
+            // P^T of query half h sits at columns 64 h .. 64 h + 31 (16-bit pairs)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8, mDOs + kk * 128u, C::IDESC_KM,
-                       (s > 0 || kk > 0) ? 1u : 0u);
+                mma_ts(tmem + C::T_DV, tmem + C::T_S + (kk >> 2) * 64 + (kk & 3) * 8, mDOs + kk * 128u,
+                       C::IDESC_KM, (s > 0 || kk > 0) ? 1u : 0u);
             mma_commit(bar(C::B_DO_EMPTY + st));
             // next S^T as soon as P^T has been consumed (in-order tensor pipe)
             const int nst = (it + 1) & 1;
@@ -461,21 +482,22 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32
                 mma_kk(C::T_S, kK, kQ + nst * STAGE);
                 mma_commit(bar(C::B_S_FULL));
             }
-            // dK += dS^T Q ; dQ^T = K^T dS^T
+            // dQ^T = K^T dS^T first (head dims on the TMEM lanes, both operands
+            // MN-major), so its drain -- which gates the next dP^T -- overlaps dK
             if (!wait_fast(bar(C::B_DS_FULL), it & 1u, ctl, W_BWD_DS_FULL)) return;
             tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + C::T_DP, mK + kk * 128u, mDS + kk * 128u, C::IDESC_MM, kk > 0 ? 1u : 0u);
+            mma_commit(bar(C::B_DQ_FULL));
+            ++dq_issued;
+            // dK += dS^T Q
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t off = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
                 mma_ss(tmem + C::T_DK, kDS + off, mQs + kk * 128u, C::IDESC_KM,
                        (s > 0 || kk > 0) ? 1u : 0u);
             }
-            // dQ^T = K^T dS^T: head dims on the TMEM lanes (both operands MN-major)
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + C::T_DP, mK + kk * 128u, mDS + kk * 128u, C::IDESC_MM, kk > 0 ? 1u : 0u);
-            mma_commit(bar(C::B_DQ_FULL));
-            ++dq_issued;
             mma_commit(bar(C::B_Q_EMPTY + st));
             mma_commit(bar(C::B_DS_EMPTY));
             // next dP^T once the dQ readers have drained TMEM
@@ -586,8 +608,8 @@ __global__ void __launch_bounds__(BwdCfg<BF16>::THREADS, 1)
         }
         mbar_init(bar(C::B_S_FULL), 1);
         mbar_init(bar(C::B_DP_FULL), 1);
-        mbar_init(bar(C::B_P_FULL), 4);
-        mbar_init(bar(C::B_DS_FULL), 4);
+        mbar_init(bar(C::B_P_FULL), 8);
+        mbar_init(bar(C::B_DS_FULL), 8);
         mbar_init(bar(C::B_DS_EMPTY), 1);
         mbar_init(bar(C::B_DQ_FULL), 1);
         mbar_init(bar(C::B_DQ_EMPTY), 4);
@@ -611,10 +633,10 @@ __global__ void __launch_bounds__(BwdCfg<BF16>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
 
-    if (warp < 4) {
-        bwd_compute<BF16>(p, tmem, base + C::OFF_DS, base + C::OFF_ROWS, bars, ctl, warp);
-    } else if (warp < 8) {
-        bwd_dq_reduce<BF16>(p, tmem, bars, ctl, warp - 4);
+    if (warp < C::DQ_WARP) {
+        bwd_compute<BF16>(p, tmem, base + C::OFF_DS, base + C::OFF_ROWS, bars, ctl, warp & 3, warp >> 2);
+    } else if (warp < C::MMA_WARP) {
+        bwd_dq_reduce<BF16>(p, tmem, bars, ctl, warp - C::DQ_WARP);
     } else if (warp == C::MMA_WARP) {
         if (lane == 0) {
             bwd_mma<BF16>(p, tmem, base, bars, ctl);

@@ -12,10 +12,11 @@
 //     key-side accumulators are kept transposed, dV^T += dO^T P and dK^T += Q^T dS,
 //     as two M = 128 head-dim halves each, reading dO, Q (MN-major) and P, dS
 //     (MN-major) straight from the tiles already in shared memory;
-//   * dQ = dS K is produced in two 128-column halves into one TMEM region, each drained
-//     by the dQ warpgroup into the fp32 accumulator with vector reductions.
+//   * dQ is produced transposed, dQ^T = K^T dS^T, in two 128-dim halves into one TMEM
+//     region (head dims on the lanes), each drained by the dQ warpgroup into the fp32
+//     accumulator, one 128-byte segment per warp-wide reduction.
 //
-// TMEM: S [0,64) | dP [64,128) | dQ half [128,256) | dV^T halves [256,384) | dK^T [384,512)
+// TMEM: S [0,64) | dP [64,128) | dQ^T half [128,256) | dV^T halves [256,384) | dK^T [384,512)
 #pragma once
 
 #include "fa_bwd.cuh"
@@ -49,7 +50,7 @@ struct Bwd256Cfg {
     static constexpr uint32_t T_S = 0, T_DP = 64, T_DQ = 128, T_DV = 256, T_DK = 384;
     static constexpr uint32_t IDESC_S = idesc_f16(BF16, 128, 64, false, false);   // S, dP
     static constexpr uint32_t IDESC_T = idesc_f16(BF16, 128, 64, true, true);     // dV^T, dK^T
-    static constexpr uint32_t IDESC_Q = idesc_f16(BF16, 128, 128, false, true);   // dQ half
+    static constexpr uint32_t IDESC_Q = idesc_f16(BF16, 128, 128, true, false);   // dQ^T half
 };
 
 enum : uint32_t {
@@ -138,13 +139,9 @@ __device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base,
                 const uint32_t a = c < 32 ? r0[c] : r1[c - 32];
                 const uint32_t b = c < 32 ? r0[c + 1] : r1[c - 31];
                 const float2 x = f2unpack(ffma2(f2pack(__uint_as_float(a), __uint_as_float(b)), sl2x2, negl2));
-                float e0, e1;
-                if (!masked && (c & 2)) {
-                    exp2_fma_x2(x.x, x.y, e0, e1);
-                } else {
-                    e0 = ex2_sfu(x.x);
-                    e1 = ex2_sfu(x.y);
-                }
+                // all on the SFU (one warp per sub-partition here: nothing hides the
+                // longer FMA-pipe sequence)
+                float e0 = ex2_sfu(x.x), e1 = ex2_sfu(x.y);
                 if (masked) {
                     if (c > lim) e0 = 0.0f;
                     if (c + 1 > lim) e1 = 0.0f;
@@ -218,13 +215,13 @@ __device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base,
     }
 }
 
-// ---- dQ warpgroup: two 128-column halves per step -> fp32 vector reductions ----------
+// ---- dQ warpgroup: two 128-dim halves of dQ^T per step -> fp32 reductions -----------
 template <bool BF16>
 __device__ void bwd256_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int wq)
 {
     using C = Bwd256Cfg<BF16>;
     const int lane = threadIdx.x & 31;
-    const int t = wq * 32 + lane;
+    const int t = wq * 32 + lane;  // head dim within the half (= TMEM lane of dQ^T)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     auto bar = [&](int i) { return bars + 8u * i; };
     uint32_t k = 0;  // dQ halves drained so far
@@ -233,22 +230,20 @@ __device__ void bwd256_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bar
         for (int s = 0; s < u.T; ++s) {
             int h, m;
             bwd_step(p, u, s, h, m);
-            float* row = p.dqacc + ((static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + m * 128 + t) * C::D;
+            float* blk = p.dqacc + ((static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + m * 128) * C::D + t;
 #pragma unroll 1
             for (int dh = 0; dh < 2; ++dh, ++k) {
                 if (!warp_wait(bar(C::B_DQ_FULL), k & 1u, ctl, W_B256_DQ_FULL)) return;
                 tc_fence_after();
-                uint32_t r[128];
+                uint32_t r[128];  // r[i] = dQ^T[dim dh*128 + t][query i]
                 tmem_ld128_wait(tmem + lane_off + C::T_DQ, r);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
-                float* dst = row + dh * 128;
+                float* dst = blk + dh * 128;
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * c),
-                                 "f"(__uint_as_float(r[4 * c])), "f"(__uint_as_float(r[4 * c + 1])),
-                                 "f"(__uint_as_float(r[4 * c + 2])), "f"(__uint_as_float(r[4 * c + 3]))
+                for (int i = 0; i < 128; ++i)
+                    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst + i * C::D), "f"(__uint_as_float(r[i]))
                                  : "memory");
             }
         }
@@ -289,11 +284,12 @@ __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uin
                 mma_ss(tmem + d_t + hf * 64, x + ((2 * hf * C::Q_BLK + kk * 2048u) >> 4), z + kk * 128u,
                        C::IDESC_T, (acc || kk > 0) ? 1u : 0u);
     };
-    // dQ half `dh` = dS K[:, 128 dh .. 128 dh + 127]
+    // dQ^T half `dh` = K[:, 128 dh .. 128 dh + 127]^T dS^T: A = K read MN-major (dims
+    // contiguous), B = the [query][key] dS tile read K-major
     auto mma_dq = [&](int dh) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + C::T_DQ, kDS + kk * 2u, mK + ((2 * dh * C::KV_BLK + kk * 2048u) >> 4), C::IDESC_Q,
+            mma_ss(tmem + C::T_DQ, mK + ((2 * dh * C::KV_BLK + kk * 2048u) >> 4), kDS + kk * 2u, C::IDESC_Q,
                    kk > 0);
     };
     auto wait_dq_free = [&]() -> bool {
