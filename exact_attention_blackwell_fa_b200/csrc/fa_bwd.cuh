@@ -156,6 +156,9 @@ struct BwdCfg {
     // warps 0-7: compute (two warpgroups, one per 64-query half), 8-11: dQ, 12: MMA, 13: TMA
     static constexpr int THREADS = 448;
     static constexpr int DQ_WARP = 8, MMA_WARP = 12, LOAD_WARP = 13;
+    // lane 0 of the MMA warp issues alone (the converged, elected-lane form measured
+    // slower here)
+    static constexpr bool WARP_ISSUE = false;
     static constexpr uint32_t TILE = 32768;  // 128 rows x 128 columns x 2 bytes
     // per query block: LSE*log2(e) and D for its 128 rows, staged with the Q tile
     static constexpr uint32_t ROWS_BYTES = 1024;
@@ -419,6 +422,7 @@ template <bool BF16>
 __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars, CtaCtl* ctl)
 {
     using C = BwdCfg<BF16>;
+    using I = Issuer<C::WARP_ISSUE>;
     auto bar = [&](int i) { return bars + 8u * i; };
     uint32_t it = 0, unit_it = 0, dq_issued = 0;
     // Descriptors are built once; each MMA adds a constant byte offset / 16 to the
@@ -438,79 +442,79 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
-            mma_ss(tmem + d_t, a + off, b + off, C::IDESC_KK, kk > 0);
+            I::ss(tmem + d_t, a + off, b + off, C::IDESC_KK, kk > 0);
         }
     };
     auto wait_dq_free = [&]() -> bool {
         if (dq_issued == 0) return true;
-        return wait_fast(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_BWD_DQ_EMPTY);
+        return I::wait(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_BWD_DQ_EMPTY);
     };
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
         const BwdUnit u = bwd_decode(p, ui);
         if (u.T == 0) continue;
-        if (!wait_fast(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_BWD_KV_FULL)) return;
+        if (!I::wait(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_BWD_KV_FULL)) return;
         tc_fence_after();
         {
             const int st = it & 1;
-            if (!wait_fast(bar(C::B_Q_FULL + st), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
+            if (!I::wait(bar(C::B_Q_FULL + st), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
             tc_fence_after();
             mma_kk(C::T_S, kK, kQ + st * STAGE);
-            mma_commit(bar(C::B_S_FULL));
+            I::commit(bar(C::B_S_FULL));
             if (!wait_dq_free()) return;
-            if (!wait_fast(bar(C::B_DO_FULL + st), (it >> 1) & 1u, ctl, W_BWD_DO_FULL)) return;
+            if (!I::wait(bar(C::B_DO_FULL + st), (it >> 1) & 1u, ctl, W_BWD_DO_FULL)) return;
             tc_fence_after();
             mma_kk(C::T_DP, kV, kDO + st * STAGE);
-            mma_commit(bar(C::B_DP_FULL));
+            I::commit(bar(C::B_DP_FULL));
         }
         for (int s = 0; s < u.T; ++s, ++it) {
             const int st = it & 1;
             const uint64_t mQs = mQ + st * STAGE, mDOs = mDO + st * STAGE;
             // dV += P^T dO
-            if (!wait_fast(bar(C::B_P_FULL), it & 1u, ctl, W_BWD_P_FULL)) return;
+            if (!I::wait(bar(C::B_P_FULL), it & 1u, ctl, W_BWD_P_FULL)) return;
             tc_fence_after();
             // P^T of query half h sits at columns 64 h .. 64 h + 31 (16-bit pairs)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ts(tmem + C::T_DV, tmem + C::T_S + (kk >> 2) * 64 + (kk & 3) * 8, mDOs + kk * 128u,
+                I::ts(tmem + C::T_DV, tmem + C::T_S + (kk >> 2) * 64 + (kk & 3) * 8, mDOs + kk * 128u,
                        C::IDESC_KM, (s > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(bar(C::B_DO_EMPTY + st));
+            I::commit(bar(C::B_DO_EMPTY + st));
             // next S^T as soon as P^T has been consumed (in-order tensor pipe)
             const int nst = (it + 1) & 1;
             if (s + 1 < u.T) {
-                if (!wait_fast(bar(C::B_Q_FULL + nst), ((it + 1) >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
+                if (!I::wait(bar(C::B_Q_FULL + nst), ((it + 1) >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
                 tc_fence_after();
                 mma_kk(C::T_S, kK, kQ + nst * STAGE);
-                mma_commit(bar(C::B_S_FULL));
+                I::commit(bar(C::B_S_FULL));
             }
             // dQ^T = K^T dS^T first (head dims on the TMEM lanes, both operands
             // MN-major), so its drain -- which gates the next dP^T -- overlaps dK
-            if (!wait_fast(bar(C::B_DS_FULL), it & 1u, ctl, W_BWD_DS_FULL)) return;
+            if (!I::wait(bar(C::B_DS_FULL), it & 1u, ctl, W_BWD_DS_FULL)) return;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + C::T_DP, mK + kk * 128u, mDS + kk * 128u, C::IDESC_MM, kk > 0 ? 1u : 0u);
-            mma_commit(bar(C::B_DQ_FULL));
+                I::ss(tmem + C::T_DP, mK + kk * 128u, mDS + kk * 128u, C::IDESC_MM, kk > 0 ? 1u : 0u);
+            I::commit(bar(C::B_DQ_FULL));
             ++dq_issued;
             // dK += dS^T Q
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t off = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
-                mma_ss(tmem + C::T_DK, kDS + off, mQs + kk * 128u, C::IDESC_KM,
+                I::ss(tmem + C::T_DK, kDS + off, mQs + kk * 128u, C::IDESC_KM,
                        (s > 0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit(bar(C::B_Q_EMPTY + st));
-            mma_commit(bar(C::B_DS_EMPTY));
+            I::commit(bar(C::B_Q_EMPTY + st));
+            I::commit(bar(C::B_DS_EMPTY));
             // next dP^T once the dQ readers have drained TMEM
             if (s + 1 < u.T) {
                 if (!wait_dq_free()) return;
-                if (!wait_fast(bar(C::B_DO_FULL + nst), ((it + 1) >> 1) & 1u, ctl, W_BWD_DO_FULL)) return;
+                if (!I::wait(bar(C::B_DO_FULL + nst), ((it + 1) >> 1) & 1u, ctl, W_BWD_DO_FULL)) return;
                 tc_fence_after();
                 mma_kk(C::T_DP, kV, kDO + nst * STAGE);
-                mma_commit(bar(C::B_DP_FULL));
+                I::commit(bar(C::B_DP_FULL));
             }
         }
-        mma_commit(bar(C::B_KV_EMPTY));
-        mma_commit(bar(C::B_DKV_FINAL));
+        I::commit(bar(C::B_KV_EMPTY));
+        I::commit(bar(C::B_DKV_FINAL));
         ++unit_it;
     }
 }
@@ -638,10 +642,10 @@ __global__ void __launch_bounds__(BwdCfg<BF16>::THREADS, 1)
     } else if (warp < C::MMA_WARP) {
         bwd_dq_reduce<BF16>(p, tmem, bars, ctl, warp - C::DQ_WARP);
     } else if (warp == C::MMA_WARP) {
-        if (lane == 0) {
+        if (C::WARP_ISSUE || lane == 0) {
             bwd_mma<BF16>(p, tmem, base, bars, ctl);
-            mma_commit(bars + 8u * C::B_DRAIN);
-            drain_wait(bars + 8u * C::B_DRAIN, 0u, W_BWD_DRAIN);
+            Issuer<C::WARP_ISSUE>::commit(bars + 8u * C::B_DRAIN);
+            if (lane == 0) drain_wait(bars + 8u * C::B_DRAIN, 0u, W_BWD_DRAIN);
         }
         __syncwarp();
     } else if (warp == C::LOAD_WARP) {

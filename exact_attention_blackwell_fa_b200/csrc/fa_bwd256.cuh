@@ -30,6 +30,9 @@ struct Bwd256Cfg {
     static constexpr int BM = 128;  // query rows per step
     static constexpr int THREADS = 384;
     static constexpr int MMA_WARP = 8, LOAD_WARP = 9;
+    // lane 0 of the MMA warp issues alone (the converged, elected-lane form measured
+    // slower here)
+    static constexpr bool WARP_ISSUE = false;
     static constexpr uint32_t KV_BLK = BN * 128;   // [64 rows][64 cols] of 16-bit values
     static constexpr uint32_t KV_BYTES = 4 * KV_BLK;
     static constexpr uint32_t Q_BLK = BM * 128;    // [128 rows][64 cols]
@@ -255,6 +258,7 @@ template <bool BF16>
 __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars, CtaCtl* ctl)
 {
     using C = Bwd256Cfg<BF16>;
+    using I = Issuer<C::WARP_ISSUE>;
     auto bar = [&](int i) { return bars + 8u * i; };
     const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQ = base + C::OFF_Q,
                    sDO = base + C::OFF_DO, sP = base + C::OFF_P, sDS = base + C::OFF_DS;
@@ -271,7 +275,7 @@ __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uin
         for (int kk = 0; kk < 16; ++kk) {
             const uint32_t xo = ((kk >> 2) * C::Q_BLK + (kk & 3) * 32u) >> 4;
             const uint32_t yo = ((kk >> 2) * C::KV_BLK + (kk & 3) * 32u) >> 4;
-            mma_ss(tmem + d_t, x + xo, y + yo, C::IDESC_S, kk > 0);
+            I::ss(tmem + d_t, x + xo, y + yo, C::IDESC_S, kk > 0);
         }
     };
     // acc^T[half] (+)= X^T Z: X a [128 query][256] tile read MN-major (head-dim half
@@ -281,7 +285,7 @@ __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uin
         for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + d_t + hf * 64, x + ((2 * hf * C::Q_BLK + kk * 2048u) >> 4), z + kk * 128u,
+                I::ss(tmem + d_t + hf * 64, x + ((2 * hf * C::Q_BLK + kk * 2048u) >> 4), z + kk * 128u,
                        C::IDESC_T, (acc || kk > 0) ? 1u : 0u);
     };
     // dQ^T half `dh` = K[:, 128 dh .. 128 dh + 127]^T dS^T: A = K read MN-major (dims
@@ -289,60 +293,60 @@ __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uin
     auto mma_dq = [&](int dh) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + C::T_DQ, mK + ((2 * dh * C::KV_BLK + kk * 2048u) >> 4), kDS + kk * 2u, C::IDESC_Q,
+            I::ss(tmem + C::T_DQ, mK + ((2 * dh * C::KV_BLK + kk * 2048u) >> 4), kDS + kk * 2u, C::IDESC_Q,
                    kk > 0);
     };
     auto wait_dq_free = [&]() -> bool {
         if (dq_issued == 0) return true;
-        return wait_fast(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_B256_DQ_EMPTY);
+        return I::wait(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_B256_DQ_EMPTY);
     };
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
         const BwdUnit u = bwd256_decode(p, ui);
         if (u.T == 0) continue;
-        if (!wait_fast(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_B256_KV_FULL)) return;
+        if (!I::wait(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_B256_KV_FULL)) return;
         tc_fence_after();
-        if (!wait_fast(bar(C::B_Q_FULL), it & 1u, ctl, W_B256_Q_FULL)) return;
+        if (!I::wait(bar(C::B_Q_FULL), it & 1u, ctl, W_B256_Q_FULL)) return;
         tc_fence_after();
         mma_qk(C::T_S, kQ, kK);
-        mma_commit(bar(C::B_S_FULL));
-        if (!wait_fast(bar(C::B_DO_FULL), it & 1u, ctl, W_B256_DO_FULL)) return;
+        I::commit(bar(C::B_S_FULL));
+        if (!I::wait(bar(C::B_DO_FULL), it & 1u, ctl, W_B256_DO_FULL)) return;
         tc_fence_after();
         mma_qk(C::T_DP, kDO, kV);
-        mma_commit(bar(C::B_DP_FULL));
+        I::commit(bar(C::B_DP_FULL));
         for (int s = 0; s < u.T; ++s, ++it) {
-            if (!wait_fast(bar(C::B_P_FULL), it & 1u, ctl, W_B256_P_FULL)) return;
+            if (!I::wait(bar(C::B_P_FULL), it & 1u, ctl, W_B256_P_FULL)) return;
             tc_fence_after();
             mma_t(C::T_DV, mDO, mP, s > 0);
-            mma_commit(bar(C::B_P_EMPTY));
-            mma_commit(bar(C::B_DO_EMPTY));
-            if (!wait_fast(bar(C::B_DS_FULL), it & 1u, ctl, W_B256_DS_FULL)) return;
+            I::commit(bar(C::B_P_EMPTY));
+            I::commit(bar(C::B_DO_EMPTY));
+            if (!I::wait(bar(C::B_DS_FULL), it & 1u, ctl, W_B256_DS_FULL)) return;
             tc_fence_after();
             mma_t(C::T_DK, mQ, mDS, s > 0);
-            mma_commit(bar(C::B_Q_EMPTY));
+            I::commit(bar(C::B_Q_EMPTY));
             if (!wait_dq_free()) return;
             tc_fence_after();
             mma_dq(0);
-            mma_commit(bar(C::B_DQ_FULL));
+            I::commit(bar(C::B_DQ_FULL));
             ++dq_issued;
             if (s + 1 < u.T) {
-                if (!wait_fast(bar(C::B_Q_FULL), (it + 1) & 1u, ctl, W_B256_Q_FULL)) return;
+                if (!I::wait(bar(C::B_Q_FULL), (it + 1) & 1u, ctl, W_B256_Q_FULL)) return;
                 tc_fence_after();
                 mma_qk(C::T_S, kQ, kK);
-                mma_commit(bar(C::B_S_FULL));
-                if (!wait_fast(bar(C::B_DO_FULL), (it + 1) & 1u, ctl, W_B256_DO_FULL)) return;
+                I::commit(bar(C::B_S_FULL));
+                if (!I::wait(bar(C::B_DO_FULL), (it + 1) & 1u, ctl, W_B256_DO_FULL)) return;
                 tc_fence_after();
                 mma_qk(C::T_DP, kDO, kV);
-                mma_commit(bar(C::B_DP_FULL));
+                I::commit(bar(C::B_DP_FULL));
             }
             if (!wait_dq_free()) return;
             tc_fence_after();
             mma_dq(1);
-            mma_commit(bar(C::B_DQ_FULL));
+            I::commit(bar(C::B_DQ_FULL));
             ++dq_issued;
-            mma_commit(bar(C::B_DS_EMPTY));
+            I::commit(bar(C::B_DS_EMPTY));
         }
-        mma_commit(bar(C::B_KV_EMPTY));
-        mma_commit(bar(C::B_DKV_FINAL));
+        I::commit(bar(C::B_KV_EMPTY));
+        I::commit(bar(C::B_DKV_FINAL));
         ++unit_it;
     }
 }
@@ -449,10 +453,10 @@ __global__ void __launch_bounds__(Bwd256Cfg<BF16>::THREADS, 1)
     } else if (warp < 8) {
         bwd256_dq_reduce<BF16>(p, tmem, bars, ctl, warp - 4);
     } else if (warp == C::MMA_WARP) {
-        if (lane == 0) {
+        if (C::WARP_ISSUE || lane == 0) {
             bwd256_mma<BF16>(p, tmem, base, bars, ctl);
-            mma_commit(bars + 8u * C::B_DRAIN);
-            drain_wait(bars + 8u * C::B_DRAIN, 0u, W_B256_DRAIN);
+            Issuer<C::WARP_ISSUE>::commit(bars + 8u * C::B_DRAIN);
+            if (lane == 0) drain_wait(bars + 8u * C::B_DRAIN, 0u, W_B256_DRAIN);
         }
         __syncwarp();
     } else if (warp == C::LOAD_WARP) {

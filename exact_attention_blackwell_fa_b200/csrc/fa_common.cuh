@@ -86,6 +86,33 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, CtaCtl*
     return ok != 0;
 }
 
+// MMA-issue primitives for either a warp-converged issuer (WARP: all 32 lanes call
+// them; each tcgen05 op is executed by one elected lane, which keeps descriptors
+// warp-uniform) or a single issuing thread.
+template <bool WARP>
+struct Issuer {
+    __device__ static bool wait(uint32_t bar, uint32_t parity, CtaCtl* ctl, uint32_t where)
+    {
+        if constexpr (WARP) return warp_wait(bar, parity, ctl, where);
+        else return wait_fast(bar, parity, ctl, where);
+    }
+    __device__ static void ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc)
+    {
+        if constexpr (WARP) mma_ss_w(d, a, b, idesc, acc);
+        else mma_ss(d, a, b, idesc, acc);
+    }
+    __device__ static void ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc)
+    {
+        if constexpr (WARP) mma_ts_w(d, a, b, idesc, acc);
+        else mma_ts(d, a, b, idesc, acc);
+    }
+    __device__ static void commit(uint32_t bar)
+    {
+        if constexpr (WARP) mma_commit_w(bar);
+        else mma_commit(bar);
+    }
+};
+
 // ---------------------------------------------------------------------------------
 // Packed fp32 pairs (sm_100 f32x2 arithmetic on the FMA pipe: two lanes of work per
 // instruction).  A pair lives in one 64-bit register, `lo` in the low half.

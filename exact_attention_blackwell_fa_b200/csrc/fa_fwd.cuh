@@ -365,22 +365,31 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, ui
 }
 
 // ---------------------------------------------------------------------------------
-// MMA issuer (one thread).
+// MMA issuer.  head_dim 256: the whole warp runs the issue loop, converged, and each
+// tcgen05 op is executed by one elected lane (warp-uniform descriptors, few
+// instructions per MMA).  head_dim 128: lane 0 alone runs it; with four softmax warps
+// per SM sub-partition at a 96-register budget the converged form measured slower.
 // ---------------------------------------------------------------------------------
 template <int D, bool BF16>
 struct FwdMma {
     using C = FwdCfg<D, BF16>;
+    static constexpr bool WARP_ISSUE = D == 256;
+    using I = Issuer<WARP_ISSUE>;
     uint32_t tmem, sQ, sRing, bars;
     CtaCtl* ctl;
     uint32_t seq = 0;  // ring chunk sequence number
 
     __device__ uint32_t bar(int i) const { return bars + 8u * i; }
+    __device__ bool wait(uint32_t b, uint32_t parity, uint32_t where) const { return I::wait(b, parity, ctl, where); }
+    __device__ static void ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) { I::ss(d, a, b, idesc, acc); }
+    __device__ static void ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) { I::ts(d, a, b, idesc, acc); }
+    __device__ static void commit(uint32_t b) { I::commit(b); }
     __device__ uint32_t slot(uint32_t s) const { return sRing + (s % C::NSTAGE) * C::CHUNK; }
     __device__ bool wait_full(uint32_t s)
     {
-        return wait_bar(bar(C::B_FULL + s % C::NSTAGE), (s / C::NSTAGE) & 1u, ctl, W_FWD_RING_FULL);
+        return wait(bar(C::B_FULL + s % C::NSTAGE), (s / C::NSTAGE) & 1u, W_FWD_RING_FULL);
     }
-    __device__ void release(uint32_t s) { mma_commit(bar(C::B_EMPTY + s % C::NSTAGE)); }
+    __device__ void release(uint32_t s) { commit(bar(C::B_EMPTY + s % C::NSTAGE)); }
 
     // Descriptors are built once; every MMA then only adds a constant byte offset / 16
     // to the 14-bit start-address field (it cannot carry: addresses stay below 256 KB).
@@ -410,7 +419,7 @@ struct FwdMma {
         for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t aoff = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
             const uint32_t boff = (((kk & 7) >> 2) * 16384u + (kk & 3) * 32u) >> 4;
-            mma_ss(d, qd + aoff, kd[kk >> 3] + boff, C::IDESC_S, kk > 0);
+            ss(d, qd + aoff, kd[kk >> 3] + boff, C::IDESC_S, kk > 0);
         }
     }
     // O_q (+)= P(q, sb) V, V tile in ring chunks sV .. sV + KCH - 1 (chunk c = O columns
@@ -428,7 +437,7 @@ struct FwdMma {
             const uint32_t a = tP + C::col_P(kk >> 2) + (kk & 3) * 8;
 #pragma unroll
             for (int c = 0; c < C::KCH; ++c)
-                mma_ts(tO + c * 128, a, vd[c] + (kk * 2048u >> 4), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                ts(tO + c * 128, a, vd[c] + (kk * 2048u >> 4), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
     }
     __device__ bool wait_chunks(uint32_t s0)
@@ -452,7 +461,7 @@ struct FwdMma {
             fwd_decode<C::UNIT_ROWS>(p, t, b, h, m0);
             const int n = fwd_kv_tiles<C::UNIT_ROWS>(p, m0);
             if (n == 0) continue;
-            if (!wait_bar(bar(C::B_Q_FULL), q_it & 1u, ctl, W_FWD_Q_FULL)) return;
+            if (!wait(bar(C::B_Q_FULL), q_it & 1u, W_FWD_Q_FULL)) return;
             ++q_it;
             tc_fence_after();
             if constexpr (C::NQ == 2) {
@@ -462,16 +471,16 @@ struct FwdMma {
                 if (!wait_chunks(sK)) return;
                 for (int q = 0; q < 2; ++q) {
                     issue_S(q, 0, sK);
-                    mma_commit(bar(C::B_S_FULL + q));
+                    commit(bar(C::B_S_FULL + q));
                     ++s_it[q];
                 }
                 release(sK);
-                if (n == 1) mma_commit(bar(C::B_Q_EMPTY));
+                if (n == 1) commit(bar(C::B_Q_EMPTY));
                 for (int j = 1; j < n; ++j) {
                     const uint32_t sV = seq;
                     seq += 1;
                     if (!wait_chunks(sV)) return;
-                    if (!wait_bar(bar(C::B_P_FULL + 0), p_it[0] & 1u, ctl, W_FWD_P_FULL)) return;
+                    if (!wait(bar(C::B_P_FULL + 0), p_it[0] & 1u, W_FWD_P_FULL)) return;
                     tc_fence_after();
                     issue_PV(0, 0, sV, j > 1);
                     ++p_it[0];
@@ -479,28 +488,28 @@ struct FwdMma {
                     seq += 1;
                     if (!wait_chunks(sK)) return;
                     issue_S(0, 0, sK);
-                    mma_commit(bar(C::B_S_FULL + 0));
+                    commit(bar(C::B_S_FULL + 0));
                     ++s_it[0];
-                    if (!wait_bar(bar(C::B_P_FULL + 1), p_it[1] & 1u, ctl, W_FWD_P_FULL)) return;
+                    if (!wait(bar(C::B_P_FULL + 1), p_it[1] & 1u, W_FWD_P_FULL)) return;
                     tc_fence_after();
                     issue_PV(1, 0, sV, j > 1);
                     ++p_it[1];
                     release(sV);
                     issue_S(1, 0, sK);
-                    mma_commit(bar(C::B_S_FULL + 1));
+                    commit(bar(C::B_S_FULL + 1));
                     ++s_it[1];
                     release(sK);
-                    if (j == n - 1) mma_commit(bar(C::B_Q_EMPTY));
+                    if (j == n - 1) commit(bar(C::B_Q_EMPTY));
                 }
                 const uint32_t sV = seq;
                 seq += 1;
                 if (!wait_chunks(sV)) return;
                 for (int q = 0; q < 2; ++q) {
-                    if (!wait_bar(bar(C::B_P_FULL + q), p_it[q] & 1u, ctl, W_FWD_P_FULL)) return;
+                    if (!wait(bar(C::B_P_FULL + q), p_it[q] & 1u, W_FWD_P_FULL)) return;
                     tc_fence_after();
                     issue_PV(q, 0, sV, n > 1);
                     ++p_it[q];
-                    mma_commit(bar(C::B_O_FINAL + q));
+                    commit(bar(C::B_O_FINAL + q));
                 }
                 release(sV);
             } else {
@@ -511,20 +520,20 @@ struct FwdMma {
                     if (!wait_chunks(sK)) return;
                     const int sb = s_it[0] & 1;
                     issue_S(0, sb, sK);
-                    mma_commit(bar(C::B_S_FULL + sb));
+                    commit(bar(C::B_S_FULL + sb));
                     ++s_it[0];
                     release_chunks(sK);
                 }
-                if (n <= 2) mma_commit(bar(C::B_Q_EMPTY));
+                if (n <= 2) commit(bar(C::B_Q_EMPTY));
                 for (int j = 0; j < n; ++j) {
                     const uint32_t sV = seq;
                     seq += C::KCH;
                     if (!wait_chunks(sV)) return;
                     const int sbp = p_it[0] & 1;
-                    if (!wait_bar(bar(C::B_P_FULL + sbp), (p_it[0] >> 1) & 1u, ctl, W_FWD_P_FULL)) return;
+                    if (!wait(bar(C::B_P_FULL + sbp), (p_it[0] >> 1) & 1u, W_FWD_P_FULL)) return;
                     tc_fence_after();
                     issue_PV(0, sbp, sV, j > 0);
-                    mma_commit(bar(C::B_O_DONE));
+                    commit(bar(C::B_O_DONE));
                     ++p_it[0];
                     release_chunks(sV);
                     if (j + 2 < n) {
@@ -533,13 +542,13 @@ struct FwdMma {
                         if (!wait_chunks(sK)) return;
                         const int sb = s_it[0] & 1;
                         issue_S(0, sb, sK);
-                        mma_commit(bar(C::B_S_FULL + sb));
+                        commit(bar(C::B_S_FULL + sb));
                         ++s_it[0];
                         release_chunks(sK);
-                        if (j + 2 == n - 1) mma_commit(bar(C::B_Q_EMPTY));
+                        if (j + 2 == n - 1) commit(bar(C::B_Q_EMPTY));
                     }
                 }
-                mma_commit(bar(C::B_O_FINAL));
+                commit(bar(C::B_O_FINAL));
             }
         }
     }
@@ -691,13 +700,14 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
     if (warp < C::SOFTMAX_WARPS) {
         fwd_softmax<D, BF16>(p, tmem, bars, smem_raw, ctl, warp >> 3, (warp >> 2) & 1, warp & 3);
     } else if (warp == C::CTRL_WARP) {
-        if (lane == 0) {
-            FwdMma<D, BF16> mma{tmem, sQ, sRing, bars, ctl};
+        using M = FwdMma<D, BF16>;
+        if (M::WARP_ISSUE || lane == 0) {
+            M mma{tmem, sQ, sRing, bars, ctl};
             mma.init_descs();
             mma.run(p);
-            // all MMAs issued by this thread must finish before TMEM is released
-            mma_commit(bars + 8u * C::B_DRAIN);
-            drain_wait(bars + 8u * C::B_DRAIN, 0u, W_FWD_DRAIN);
+            // all MMAs issued by this warp must finish before TMEM is released
+            M::commit(bars + 8u * C::B_DRAIN);
+            if (lane == 0) drain_wait(bars + 8u * C::B_DRAIN, 0u, W_FWD_DRAIN);
         }
         __syncwarp();
     } else if (warp == C::CTRL_WARP + 1) {
