@@ -148,19 +148,31 @@ __device__ __forceinline__ float fmax3(float a, float b, float c)
     return d;
 }
 
-// exp2_fma on a pair with packed arithmetic; same steps and constants as exp2_fma.
-__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& e0, float& e1)
+// exp2_fma on a pair: the range reduction in packed fp32 (x arrives packed), the cubic
+// in scalar FMAs with immediate coefficients (no registers held for constants), and
+// 2^n applied with one integer multiply-add per value: the bits of t = x + 1.5*2^23
+// are 0x4B400000 + n, and (t_bits * 2^23) mod 2^32 = n << 23.
+__device__ __forceinline__ uint32_t imad_u32(uint32_t a, uint32_t b, uint32_t c)
 {
-    const uint64_t x = f2pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+    uint32_t d;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ void exp2_fma_x2(uint64_t x2, float& e0, float& e1)
+{
+    const float2 xc = f2unpack(x2);
+    const uint64_t x = f2pack(fmaxf(xc.x, -126.0f), fmaxf(xc.y, -126.0f));
     const uint64_t t = fadd2(x, f2pack(12582912.0f, 12582912.0f));
     const uint64_t n = fadd2(t, f2pack(-12582912.0f, -12582912.0f));
-    const uint64_t f = ffma2(n, f2pack(-1.0f, -1.0f), x);  // x - n, exact
-    uint64_t p = ffma2(f2pack(FA_EXP2_C3, FA_EXP2_C3), f, f2pack(FA_EXP2_C2, FA_EXP2_C2));
-    p = ffma2(p, f, f2pack(FA_EXP2_C1, FA_EXP2_C1));
-    p = ffma2(p, f, f2pack(FA_EXP2_C0, FA_EXP2_C0));
-    const float2 pf = f2unpack(p), tf = f2unpack(t);
-    e0 = __int_as_float(__float_as_int(pf.x) + (__float_as_int(tf.x) << 23));
-    e1 = __int_as_float(__float_as_int(pf.y) + (__float_as_int(tf.y) << 23));
+    const float2 f = f2unpack(ffma2(n, f2pack(-1.0f, -1.0f), x));  // x - n, exact
+    float p0 = fmaf(FA_EXP2_C3, f.x, FA_EXP2_C2), p1 = fmaf(FA_EXP2_C3, f.y, FA_EXP2_C2);
+    p0 = fmaf(p0, f.x, FA_EXP2_C1);
+    p1 = fmaf(p1, f.y, FA_EXP2_C1);
+    p0 = fmaf(p0, f.x, FA_EXP2_C0);
+    p1 = fmaf(p1, f.y, FA_EXP2_C0);
+    const float2 tf = f2unpack(t);
+    e0 = __uint_as_float(imad_u32(__float_as_uint(tf.x), 1u << 23, __float_as_uint(p0)));
+    e1 = __uint_as_float(imad_u32(__float_as_uint(tf.y), 1u << 23, __float_as_uint(p1)));
 }
 
 // ---------------------------------------------------------------------------------
@@ -178,18 +190,13 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
     }
 }
 
-// Packing of P (values in [0, 2^8]) for the P V product.  bf16: round to nearest with
-// ties away from zero done with integer adds and a byte permute, which keeps the
-// conversion off the special-function pipe that the SFU exponentials already load;
-// fp16: the hardware conversion (round to nearest even).
+// Packing of P (values in [0, 2^8]) for the P V product: one conversion instruction
+// per pair (round to nearest even), measured cheaper than integer rounding and a byte
+// permute on sm_100.
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2_p(float lo, float hi)
 {
-    if constexpr (BF16) {
-        return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-    } else {
-        return pack2<false>(lo, hi);
-    }
+    return pack2<BF16>(lo, hi);
 }
 
 template <bool BF16>

@@ -17,18 +17,20 @@
 //   * one thread issues tcgen05.mma: S = Q K^T into TMEM, then O += P V with P read
 //     back from TMEM (P overwrites the first half of its own S buffer as 16-bit
 //     pairs);
-//   * two softmax warpgroups per Q tile, each owning 64 of the 128 key columns of
-//     every query row (thread = query row): they load their half of S from TMEM,
-//     apply the scale and mask, swap half-row maxima through shared memory, keep the
-//     running row max / half-row sum, rescale their half of O in TMEM only when the
-//     row max grew by more than kRescaleTau (log2 units), compute P with exp2 split
-//     between the SFU and an FMA-pipe cubic, and finally normalise and write their
-//     half of O (the halves' row sums are combined once per unit);
+//   * softmax warpgroups (thread = query row) load S from TMEM, apply the scale and
+//     mask, keep the running row max and sum, rescale O in TMEM only when the row max
+//     grew by more than kRescaleTau (log2 units), write P back into TMEM as 16-bit
+//     pairs, and finally normalise and write O and LSE.  The exp2 can be split
+//     between the SFU and an FMA-pipe cubic (FwdCfg::POLY_EVERY); on sm_100 the SFU
+//     alone measured faster for both head dims, so the split is off;
 //
-// head_dim 128: two Q tiles (256 query rows) per unit, TMEM = S0 | S1 | O0 | O1; the
-// tensor core alternates between the two tiles so that one tile's softmax overlaps
-// the other tile's MMAs.  head_dim 256: one Q tile, TMEM = S(a) | S(b) | O (256
-// columns); S is double buffered so the next S = Q K^T runs during the softmax.
+// head_dim 128: two Q tiles (256 query rows) per unit, TMEM = S0 | S1 | O0 | O1, one
+// softmax warpgroup per Q tile holding a whole 128-key row in registers; the tensor
+// core alternates between the two tiles so that one tile's softmax overlaps the
+// other tile's MMAs.  head_dim 256: one Q tile, TMEM = S(a) | S(b) | O (256
+// columns), S double buffered so the next S = Q K^T runs during the softmax; two
+// softmax warpgroups each own 64 of the 128 key columns and swap half-row maxima
+// through shared memory (speculatively: see fwd_softmax).
 #pragma once
 
 #include <type_traits>
@@ -69,12 +71,16 @@ struct FwdCfg {
     static constexpr int NSTAGE = 4;             // ring depth, in chunks
     static constexpr int BM = 128;               // query rows per Q tile
     static constexpr int BN = 128;               // keys per KV tile
-    static constexpr int HALF = 64;              // key columns per softmax warpgroup
+    // softmax warpgroups per Q tile: head_dim 128 uses one (thread = a whole 128-key
+    // row); head_dim 256 two, each owning 64 of the 128 key columns
+    static constexpr int HALVES = D == 128 ? 1 : 2;
+    static constexpr int HALF = 128 / HALVES;    // key columns per softmax warpgroup
+    static constexpr int POLY_EVERY = 0;         // exp2 pairs: 1 in POLY_EVERY on the FMA pipe (0: none)
     static constexpr int UNIT_ROWS = NQ * BM;
     static constexpr uint32_t CHUNK = 32768;
     static constexpr uint32_t QTILE = BM * D * 2;
     static constexpr uint32_t Q_BYTES = NQ * QTILE;
-    static constexpr int SOFTMAX_WARPS = NQ * 8;     // two warpgroups per Q tile
+    static constexpr int SOFTMAX_WARPS = NQ * HALVES * 4;
     static constexpr int CTRL_WARP = SOFTMAX_WARPS;  // MMA warp; the TMA warp follows it
     static constexpr int THREADS = (SOFTMAX_WARPS + 2) * 32;
 
@@ -108,6 +114,11 @@ struct FwdCfg {
     // P for key columns 64h .. 64h+63 is written by softmax half h over the first 32
     // columns of its own (already consumed) half of the S buffer
     __device__ static constexpr uint32_t col_P(int half) { return half * 64; }
+    // TMEM column of the packed P words for keys 16 kk .. 16 kk + 15
+    __device__ static constexpr uint32_t col_Pk(int kk)
+    {
+        return HALVES == 2 ? col_P(kk >> 2) + (kk & 3) * 8 : kk * 8;
+    }
 
     static constexpr uint32_t IDESC_S = idesc_f16(BF16, 128, 128, false, false);
     static constexpr uint32_t IDESC_PV = idesc_f16(BF16, 128, 128, false, true);
@@ -143,6 +154,159 @@ __device__ __forceinline__ int fwd_kv_tiles(const FwdParams& p, int m0)
 }
 
 // ---------------------------------------------------------------------------------
+// Softmax / epilogue warpgroup, one per 128-row Q tile (head_dim 128): thread = one
+// query row, all 128 key columns of a tile held in registers.
+// ---------------------------------------------------------------------------------
+template <int D, bool BF16>
+__device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int q, int wq)
+{
+    using C = FwdCfg<D, BF16>;
+    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    static_assert(C::HALVES == 1 && C::NS == 1, "row softmax: one warpgroup, one S buffer per Q tile");
+    const int lane = threadIdx.x & 31;
+    const int r_in_tile = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::col_S(q, 0);
+    const uint32_t tO = tmem + lane_off + C::col_O(q);
+    auto bar = [&](int i) { return bars + 8u * i; };
+    const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
+    uint32_t s_it = 0, tile_it = 0;
+
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+        int b, h, m0;
+        fwd_decode<C::UNIT_ROWS>(p, t, b, h, m0);
+        const int n = fwd_kv_tiles<C::UNIT_ROWS>(p, m0);
+        const int q0 = m0 + q * C::BM;  // first query row of this Q tile
+        const int row = q0 + r_in_tile;
+        const bool row_ok = row < p.Sq;
+        T* orow = reinterpret_cast<T*>(p.o) + ((static_cast<size_t>(b) * p.Sq + row) * p.Hq + h) * D;
+        float* lrow = p.lse + (static_cast<size_t>(b) * p.Hq + h) * p.Sq + row;
+        if (n == 0) {  // causal with Sq > Sk: no key is visible to any row of the unit
+            if (row_ok) {
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
+                *lrow = -INFINITY;
+            }
+            continue;
+        }
+        // columns >= lim are masked for this row; the tile-level test uses the first
+        // row of the Q tile, which has the smallest limit
+        const int lim = p.causal ? min(p.Sk, row + p.Sk - p.Sq + 1) : p.Sk;
+        const int lim0 = p.causal ? min(p.Sk, q0 + p.Sk - p.Sq + 1) : p.Sk;
+
+        float m_ref = -INFINITY;  // running reference max (log2 units)
+        float l = 0.0f;           // running row sum against m_ref
+        for (int j = 0; j < n; ++j, ++s_it) {
+            if (!warp_wait(bar(C::B_S_FULL + q), s_it & 1u, ctl, W_FWD_S_FULL)) return;
+            tc_fence_after();
+            uint32_t sr[128];
+            {
+                uint32_t (&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+                uint32_t (&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+                uint32_t (&a2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
+                uint32_t (&a3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
+                tmem_ld32_nowait(tS, a0);
+                tmem_ld32_nowait(tS + 32, a1);
+                tmem_ld32_nowait(tS + 64, a2);
+                tmem_ld32_nowait(tS + 96, a3);
+                tmem_wait_ld_dep(a0);
+                tmem_wait_ld_dep(a1);
+                tmem_wait_ld_dep(a2);
+                tmem_wait_ld_dep(a3);
+            }
+            const int c0 = j * C::BN;  // key index of column 0
+            const bool masked = c0 + C::BN > lim0;
+            if (masked) {
+                const int cut = lim - c0;
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c >= cut) sr[c] = __float_as_uint(-INFINITY);
+            }
+            float mx[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mx[i] = fmaxf(__uint_as_float(sr[i]), __uint_as_float(sr[4 + i]));
+#pragma unroll
+            for (int c = 8; c < 128; c += 8)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    mx[i] = fmax3(mx[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 4 + i]));
+            const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.sl2;  // scale > 0
+            const float m_new = fmaxf(m_ref, m_tile);
+            const bool resc = (m_ref != -INFINITY) && (m_new - m_ref > kRescaleTau);
+            const float alpha = resc ? ex2_sfu(m_ref - m_new) : 1.0f;
+            if (m_ref == -INFINITY || resc) m_ref = m_new;
+            // P = 2^(S scale log2e - m_ref), stored 32 columns at a time as 16-bit pairs
+            // over the first 64 columns of the S buffer (every S value is in registers)
+            const float negm = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+            const uint64_t negm2 = f2pack(negm, negm);
+            uint64_t acc2[2] = {f2pack(0.0f, 0.0f), f2pack(0.0f, 0.0f)};
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 32; k += 2) {
+                    const int c = cc * 32 + k;
+                    const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm2);
+                    float e0, e1;
+                    if (C::POLY_EVERY > 0 && !masked && (c >> 1) % C::POLY_EVERY == C::POLY_EVERY - 1) {
+                        exp2_fma_x2(x2, e0, e1);
+                    } else {
+                        const float2 x = f2unpack(x2);
+                        e0 = ex2_sfu(x.x);
+                        e1 = ex2_sfu(x.y);
+                    }
+                    acc2[(k >> 1) & 1] = fadd2(acc2[(k >> 1) & 1], f2pack(e0, e1));
+                    pk[k >> 1] = pack2_p<BF16>(e0, e1);
+                }
+                tmem_st16(tS + cc * 16, pk);
+            }
+            const float2 a = f2unpack(fadd2(acc2[0], acc2[1]));
+            // O holds every earlier P V product here (S_full of this tile was committed
+            // after the previous P V), so it can be rescaled before this P is released
+            if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32_wait(tO + cc * 32, r);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+                    tmem_st32(tO + cc * 32, r);
+                }
+            }
+            l = l * alpha + (a.x + a.y);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q));
+        }
+        // epilogue: wait for the unit's last P V, normalise and store O and LSE
+        if (!warp_wait(bar(C::B_O_FINAL + q), tile_it & 1u, ctl, W_FWD_O_FINAL)) return;
+        ++tile_it;
+        tc_fence_after();
+        const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld32_wait(tO + cc * 32, r);
+            uint32_t pk[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                pk[k] = pack2<BF16>(__uint_as_float(r[2 * k]) * inv, __uint_as_float(r[2 * k + 1]) * inv);
+            if (row_ok) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+                dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+            }
+        }
+        if (row_ok) *lrow = (l > 0.0f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        tc_fence_before();
+    }
+}
+
+// ---------------------------------------------------------------------------------
 // Softmax / epilogue warpgroups: two per Q tile, `half` owns key columns 64h..64h+63.
 // ---------------------------------------------------------------------------------
 template <int D, bool BF16>
@@ -159,6 +323,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, ui
     float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX) + q * (2 * 2 * C::BM);
     float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM) + q * (2 * C::BM);
     auto bar = [&](int i) { return bars + 8u * i; };
+    const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
     uint32_t s_it = 0, pv_it = 0, tile_it = 0;
 
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
@@ -264,7 +429,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, ui
             uint32_t pk[32];
             auto exp_pass = [&]() -> float {
                 const float negm = (m_ref == -INFINITY) ? 0.0f : -m_ref;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint64_t negm2 = f2pack(negm, negm);
+                uint64_t acc2[2] = {f2pack(0.0f, 0.0f), f2pack(0.0f, 0.0f)};
                 tmem_ld32_nowait(tS, r0);
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
@@ -279,22 +445,24 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, ui
                     }
 #pragma unroll
                     for (int k = 0; k < 32; k += 2) {
-                        const float x0 = fmaf(__uint_as_float(r[k]), p.sl2, negm);
-                        const float x1 = fmaf(__uint_as_float(r[k + 1]), p.sl2, negm);
+                        const uint64_t x2 =
+                            ffma2(f2pack(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), sl2x2, negm2);
                         float e0, e1;
-                        // one pair in four on the FMA pipe (packed cubic), the rest on the
-                        // SFU; masked tiles use the SFU only (it maps -inf to exactly 0)
-                        if (!masked && (k & 6) == 6) {
-                            exp2_fma_x2(x0, x1, e0, e1);
+                        // one pair in C::POLY_EVERY on the FMA pipe (cubic), the rest on
+                        // the SFU; masked tiles use the SFU only (it maps -inf to exactly 0)
+                        if (C::POLY_EVERY > 0 && !masked && (k >> 1) % C::POLY_EVERY == C::POLY_EVERY - 1) {
+                            exp2_fma_x2(x2, e0, e1);
                         } else {
-                            e0 = ex2_sfu(x0);
-                            e1 = ex2_sfu(x1);
+                            const float2 x = f2unpack(x2);
+                            e0 = ex2_sfu(x.x);
+                            e1 = ex2_sfu(x.y);
                         }
-                        acc[(k >> 1) & 3] += e0 + e1;
+                        acc2[(k >> 1) & 1] = fadd2(acc2[(k >> 1) & 1], f2pack(e0, e1));
                         pk[cc * 16 + (k >> 1)] = pack2_p<BF16>(e0, e1);
                     }
                 }
-                return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                const float2 a = f2unpack(fadd2(acc2[0], acc2[1]));
+                return a.x + a.y;
             };
             // P overwrites the first 32 columns of this half's (consumed) S columns
             auto store_p = [&]() {
@@ -367,8 +535,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, ui
 // ---------------------------------------------------------------------------------
 // MMA issuer.  head_dim 256: the whole warp runs the issue loop, converged, and each
 // tcgen05 op is executed by one elected lane (warp-uniform descriptors, few
-// instructions per MMA).  head_dim 128: lane 0 alone runs it; with four softmax warps
-// per SM sub-partition at a 96-register budget the converged form measured slower.
+// instructions per MMA).  head_dim 128: lane 0 alone runs it (the converged form
+// measured about half as fast there).
 // ---------------------------------------------------------------------------------
 template <int D, bool BF16>
 struct FwdMma {
@@ -434,7 +602,7 @@ struct FwdMma {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             // k-steps 0-3 read P of key columns 0-63 (half 0), 4-7 of 64-127 (half 1)
-            const uint32_t a = tP + C::col_P(kk >> 2) + (kk & 3) * 8;
+            const uint32_t a = tP + C::col_Pk(kk);
 #pragma unroll
             for (int c = 0; c < C::KCH; ++c)
                 ts(tO + c * 128, a, vd[c] + (kk * 2048u >> 4), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
@@ -670,7 +838,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
         }
         for (int i = 0; i < C::NQ * C::NS; ++i) {
             mbar_init(bar(C::B_S_FULL + i), 1);
-            mbar_init(bar(C::B_P_FULL + i), 8);  // one arrive per softmax warp of the tile
+            mbar_init(bar(C::B_P_FULL + i), 4 * C::HALVES);  // one arrive per softmax warp of the tile
         }
         for (int q = 0; q < C::NQ; ++q) {
             mbar_init(bar(C::B_O_DONE + q), 1);
@@ -698,7 +866,10 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
     const uint32_t tmem = ctl->tmem_base;
 
     if (warp < C::SOFTMAX_WARPS) {
-        fwd_softmax<D, BF16>(p, tmem, bars, smem_raw, ctl, warp >> 3, (warp >> 2) & 1, warp & 3);
+        if constexpr (C::HALVES == 1)
+            fwd_softmax_row<D, BF16>(p, tmem, bars, ctl, warp >> 2, warp & 3);
+        else
+            fwd_softmax<D, BF16>(p, tmem, bars, smem_raw, ctl, warp >> 3, (warp >> 2) & 1, warp & 3);
     } else if (warp == C::CTRL_WARP) {
         using M = FwdMma<D, BF16>;
         if (M::WARP_ISSUE || lane == 0) {
