@@ -41,6 +41,35 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+def kernel_source_digest():
+    """sha256 over the CUDA sources, to tell whether a recorded ncu capture still
+    describes the kernels that run."""
+    import hashlib
+    csrc = os.path.join(ROOT, "exact_attention_blackwell_fa_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from the ncu capture recorded in
+    profiles/traffic.json, or None if there is none or the sources changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    for r in rec.get("captures", []):
+        if r.get("kernel") == kernel and r.get("workload") == workload and \
+                r.get("source_sha256") == kernel_source_digest():
+            return float(r["dram_bytes_per_launch"])
+    return None
+
+
 def flops(B, Sq, Sk, H, d, causal):
     f = 4.0 * B * H * Sq * Sk * d
     if causal:
@@ -331,7 +360,8 @@ def main():
                 if do_bwd else None),
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                      "peak_kind": f"{peak_kind} sustained bf16 (cuBLAS loop)",
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None},
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic(dom, config["workload"])},
         "e2e": e2e,
         "gpu_launches": K * (1 + (3 if do_bwd else 0)),
         "clocks": clocks,
