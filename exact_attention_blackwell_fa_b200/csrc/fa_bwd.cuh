@@ -25,6 +25,7 @@
 #pragma once
 
 #include <type_traits>
+#include <utility>
 
 #include "fa_common.cuh"
 
@@ -153,9 +154,15 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p)
 template <bool BF16>
 struct BwdCfg {
     static constexpr int D = 128;
-    // warps 0-7: compute (two warpgroups, one per 64-query half), 8-11: dQ, 12: MMA, 13: TMA
-    static constexpr int THREADS = 448;
+    // warps 0-7: compute (two warpgroups, one per 64-query half), 8-11: dQ, 12: MMA,
+    // 13: TMA, 14-15: idle (they complete the fourth warpgroup for setmaxnreg)
+    static constexpr int THREADS = 512;
     static constexpr int DQ_WARP = 8, MMA_WARP = 12, LOAD_WARP = 13;
+    // registers per thread: launched at 128; the MMA/TMA warpgroup gives 24 of them to
+    // the dQ warpgroup, which then holds a whole 128-column dQ^T row in registers
+    static constexpr uint32_t REG_LAUNCH = 128, REG_DQ = 152, REG_CTRL = 104;
+    static_assert(8 * 32 * REG_LAUNCH + 4 * 32 * REG_DQ + 4 * 32 * REG_CTRL <= THREADS * REG_LAUNCH,
+                  "register split exceeds the launch budget");
     // lane 0 of the MMA warp issues alone (the converged, elected-lane form measured
     // slower here)
     static constexpr bool WARP_ISSUE = false;
@@ -247,8 +254,8 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
             const bool masked = p.causal && (u.n * 128 + 127 > m * 128 + p.Sk - p.Sq);
             const int jlim = j - (p.Sk - p.Sq) - m * 128 - q0;  // visible iff column c >= jlim
             // the Q-tile barrier also covers the staged row terms
-            if (!warp_wait(bar(C::B_Q_FULL + (it & 1)), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
-            if (!warp_wait(bar(C::B_S_FULL), it & 1u, ctl, W_BWD_S_FULL)) return;
+            if (!warp_wait<true>(bar(C::B_Q_FULL + (it & 1)), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
+            if (!warp_wait<true>(bar(C::B_S_FULL), it & 1u, ctl, W_BWD_S_FULL)) return;
             tc_fence_after();
             // P^T = 2^(S^T scale log2e - LSE log2e), 32 query columns at a time.  The
             // 16-bit P^T words stay in registers for dS: the MMA issues the next S^T into
@@ -294,8 +301,8 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
             if (lane == 0) mbar_arrive(bar(C::B_P_FULL));
 
             // dS^T = P^T (dP^T - D), 32 query columns at a time (next chunk's load in flight)
-            if (!warp_wait(bar(C::B_DP_FULL), it & 1u, ctl, W_BWD_DP_FULL)) return;
-            if (!warp_wait(bar(C::B_DS_EMPTY), (it & 1u) ^ 1u, ctl, W_BWD_DS_EMPTY)) return;
+            if (!warp_wait<true>(bar(C::B_DP_FULL), it & 1u, ctl, W_BWD_DP_FULL)) return;
+            if (!warp_wait<true>(bar(C::B_DS_EMPTY), (it & 1u) ^ 1u, ctl, W_BWD_DS_EMPTY)) return;
             tc_fence_after();
             tmem_ld32_nowait(tDP, rbuf[0]);
 #pragma unroll
@@ -335,7 +342,7 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
             if (lane == 0) mbar_arrive(bar(C::B_DS_FULL));
         }
         // epilogue: dV and dK rows of this key block
-        if (!warp_wait(bar(C::B_DKV_FINAL), unit_it & 1u, ctl, W_BWD_DKV_FINAL)) return;
+        if (!warp_wait<true>(bar(C::B_DKV_FINAL), unit_it & 1u, ctl, W_BWD_DKV_FINAL)) return;
         ++unit_it;
         tc_fence_after();
         const bool row_ok = j < p.Sk;
@@ -368,6 +375,19 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
     }
 }
 
+// dst[i * STRIDE bytes] += r[i] for every i, from one base address with immediate
+// offsets (no per-row address registers)
+template <int OFF>
+__device__ __forceinline__ void red_at(float* dst, uint32_t v)
+{
+    asm volatile("red.global.add.f32 [%0+%2], %1;" ::"l"(dst), "f"(__uint_as_float(v)), "n"(OFF) : "memory");
+}
+template <int STRIDE, size_t... I>
+__device__ __forceinline__ void red_rows(float* dst, const uint32_t (&r)[sizeof...(I)], std::index_sequence<I...>)
+{
+    (red_at<static_cast<int>(I) * STRIDE>(dst, r[I]), ...);
+}
+
 // ---- dQ warpgroup: TMEM -> registers -> fp32 vector reductions ----------------------
 template <bool BF16>
 __device__ void bwd_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int wq)
@@ -383,36 +403,32 @@ __device__ void bwd_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, 
         for (int s = 0; s < u.T; ++s, ++it) {
             int h, m;
             bwd_step(p, u, s, h, m);
-            if (!warp_wait(bar(C::B_DQ_FULL), it & 1u, ctl, W_BWD_DQ_FULL)) return;
+            if (!warp_wait<true>(bar(C::B_DQ_FULL), it & 1u, ctl, W_BWD_DQ_FULL)) return;
             tc_fence_after();
-            // lanes hold consecutive dims, so each warp-wide reduction covers 128
-            // contiguous bytes of one accumulator row.  Two 64-query halves (the
-            // register budget of this 14-warp block); TMEM is released after the
-            // second half has been read, the first half's reductions already issued.
-            float* dst = p.dqacc + ((static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + m * 128) * C::D + t;
-#pragma unroll
-            for (int hq = 0; hq < 2; ++hq) {
-                uint32_t r0[32], r1[32];  // dQ^T[dim t][query 64 hq + i]
-                tmem_ld32_nowait(tmem + lane_off + C::T_DP + hq * 64, r0);
-                tmem_ld32_nowait(tmem + lane_off + C::T_DP + hq * 64 + 32, r1);
-                tmem_wait_ld_dep(r0);
-                tmem_wait_ld_dep(r1);
-                if (hq == 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
-                }
-                float* d0 = dst + hq * 64 * C::D;
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(d0 + i * C::D), "f"(__uint_as_float(r0[i]))
-                                 : "memory");
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(d0 + (32 + i) * C::D),
-                                 "f"(__uint_as_float(r1[i]))
-                                 : "memory");
+            // the whole dQ^T row of this thread's head dim, then TMEM is released (the
+            // next dP^T waits for it) before any reduction is issued
+            uint32_t r[128];  // r[i] = dQ^T[dim t][query i] of this block
+            {
+                uint32_t (&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+                uint32_t (&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+                uint32_t (&a2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
+                uint32_t (&a3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
+                tmem_ld32_nowait(tmem + lane_off + C::T_DP, a0);
+                tmem_ld32_nowait(tmem + lane_off + C::T_DP + 32, a1);
+                tmem_ld32_nowait(tmem + lane_off + C::T_DP + 64, a2);
+                tmem_ld32_nowait(tmem + lane_off + C::T_DP + 96, a3);
+                tmem_wait_ld_dep(a0);
+                tmem_wait_ld_dep(a1);
+                tmem_wait_ld_dep(a2);
+                tmem_wait_ld_dep(a3);
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
+            // lanes hold consecutive dims, so each warp-wide reduction covers 128
+            // contiguous bytes of one accumulator row
+            float* dst = p.dqacc + ((static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + m * 128) * C::D + t;
+            red_rows<C::D * 4>(dst, r, std::make_index_sequence<128>{});
         }
     }
 }
@@ -422,7 +438,7 @@ template <bool BF16>
 __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars, CtaCtl* ctl)
 {
     using C = BwdCfg<BF16>;
-    using I = Issuer<C::WARP_ISSUE>;
+    using I = Issuer<C::WARP_ISSUE, true>;
     auto bar = [&](int i) { return bars + 8u * i; };
     uint32_t it = 0, unit_it = 0, dq_issued = 0;
     // Descriptors are built once; each MMA adds a constant byte offset / 16 to the
@@ -542,7 +558,7 @@ struct BwdLoad {
         for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
             const BwdUnit u = bwd_decode(p, ui);
             if (u.T == 0) continue;
-            if (!wait_bar(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_BWD_KV_EMPTY)) return;
+            if (!wait_bar_inl(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_BWD_KV_EMPTY)) return;
             mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::TILE);
             tile(base + C::OFF_K, tmK, bar(C::B_KV_FULL), u.hkv, u.n * 128, u.b);
             tile(base + C::OFF_V, tmV, bar(C::B_KV_FULL), u.hkv, u.n * 128, u.b);
@@ -553,7 +569,7 @@ struct BwdLoad {
                 bwd_step(p, u, s, h, m);
                 const int st = it & 1;
                 const uint32_t ph = ((it >> 1) & 1u) ^ 1u;
-                if (!wait_bar(bar(C::B_Q_EMPTY + st), ph, ctl, W_BWD_Q_EMPTY)) return;
+                if (!wait_bar_inl(bar(C::B_Q_EMPTY + st), ph, ctl, W_BWD_Q_EMPTY)) return;
                 mbar_arrive_expect_tx(bar(C::B_Q_FULL + st), C::TILE + C::ROWS_BYTES);
                 tile(base + C::OFF_Q + st * C::TILE, tmQ, bar(C::B_Q_FULL + st), h, m * 128, u.b);
                 {
@@ -564,7 +580,7 @@ struct BwdLoad {
                     bulk_load(dst + 512, p.Dv + rb, 512, bar(C::B_Q_FULL + st));
                 }
                 q_round[st] = static_cast<int>(it >> 1);
-                if (!wait_bar(bar(C::B_DO_EMPTY + st), ph, ctl, W_BWD_DO_EMPTY)) return;
+                if (!wait_bar_inl(bar(C::B_DO_EMPTY + st), ph, ctl, W_BWD_DO_EMPTY)) return;
                 mbar_arrive_expect_tx(bar(C::B_DO_FULL + st), C::TILE);
                 tile(base + C::OFF_DO + st * C::TILE, tmDO, bar(C::B_DO_FULL + st), h, m * 128, u.b);
                 do_round[st] = static_cast<int>(it >> 1);
@@ -573,10 +589,10 @@ struct BwdLoad {
     }
     __device__ void drain()
     {
-        if (kv_round >= 0) drain_wait(bar(C::B_KV_FULL), static_cast<uint32_t>(kv_round) & 1u, W_BWD_DRAIN);
+        if (kv_round >= 0) drain_wait_inl(bar(C::B_KV_FULL), static_cast<uint32_t>(kv_round) & 1u, W_BWD_DRAIN);
         for (int st = 0; st < 2; ++st) {
-            if (q_round[st] >= 0) drain_wait(bar(C::B_Q_FULL + st), static_cast<uint32_t>(q_round[st]) & 1u, W_BWD_DRAIN);
-            if (do_round[st] >= 0) drain_wait(bar(C::B_DO_FULL + st), static_cast<uint32_t>(do_round[st]) & 1u, W_BWD_DRAIN);
+            if (q_round[st] >= 0) drain_wait_inl(bar(C::B_Q_FULL + st), static_cast<uint32_t>(q_round[st]) & 1u, W_BWD_DRAIN);
+            if (do_round[st] >= 0) drain_wait_inl(bar(C::B_DO_FULL + st), static_cast<uint32_t>(do_round[st]) & 1u, W_BWD_DRAIN);
         }
     }
 };
@@ -636,25 +652,30 @@ __global__ void __launch_bounds__(BwdCfg<BF16>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
-
+    // register split (setmaxnreg, per warpgroup): warps 12-15 release registers on entry
+    // to their branch, unconditionally, so the dQ warpgroup's increase always completes
     if (warp < C::DQ_WARP) {
         bwd_compute<BF16>(p, tmem, base + C::OFF_DS, base + C::OFF_ROWS, bars, ctl, warp & 3, warp >> 2);
     } else if (warp < C::MMA_WARP) {
+        setmaxnreg_inc<C::REG_DQ>();  // completes once warps 12-15 have released theirs
         bwd_dq_reduce<BF16>(p, tmem, bars, ctl, warp - C::DQ_WARP);
-    } else if (warp == C::MMA_WARP) {
-        if (C::WARP_ISSUE || lane == 0) {
-            bwd_mma<BF16>(p, tmem, base, bars, ctl);
-            Issuer<C::WARP_ISSUE>::commit(bars + 8u * C::B_DRAIN);
-            if (lane == 0) drain_wait(bars + 8u * C::B_DRAIN, 0u, W_BWD_DRAIN);
+    } else {
+        setmaxnreg_dec<C::REG_CTRL>();  // all four warps, first thing, unconditionally
+        if (warp == C::MMA_WARP) {
+            if (C::WARP_ISSUE || lane == 0) {
+                bwd_mma<BF16>(p, tmem, base, bars, ctl);
+                Issuer<C::WARP_ISSUE, true>::commit(bars + 8u * C::B_DRAIN);
+                if (lane == 0) drain_wait_inl(bars + 8u * C::B_DRAIN, 0u, W_BWD_DRAIN);
+            }
+            __syncwarp();
+        } else if (warp == C::LOAD_WARP) {
+            if (lane == 0) {
+                BwdLoad<BF16> ld{&tmQ, &tmK, &tmV, &tmDO, base, bars, ctl};
+                ld.run(p);
+                ld.drain();
+            }
+            __syncwarp();
         }
-        __syncwarp();
-    } else if (warp == C::LOAD_WARP) {
-        if (lane == 0) {
-            BwdLoad<BF16> ld{&tmQ, &tmK, &tmV, &tmDO, base, bars, ctl};
-            ld.run(p);
-            ld.drain();
-        }
-        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();

@@ -34,7 +34,9 @@ __device__ __forceinline__ void record_timeout(uint32_t where)
 
 // Single-thread bounded wait.  Returns false (and raises the CTA abort flag) if the
 // phase did not complete within kWaitTimeoutNs, or if another wait already aborted.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, CtaCtl* ctl, uint32_t where)
+// The _inl forms are for kernels that change per-warpgroup register budgets
+// (setmaxnreg): their code may not call out-of-line functions.
+__device__ __forceinline__ bool wait_bar_inl(uint32_t bar, uint32_t parity, CtaCtl* ctl, uint32_t where)
 {
     if (mbar_try_wait(bar, parity)) return true;
     volatile uint32_t* abort = &ctl->abort;
@@ -52,9 +54,14 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, CtaCtl* ctl
     }
 }
 
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, CtaCtl* ctl, uint32_t where)
+{
+    return wait_bar_inl(bar, parity, ctl, where);
+}
+
 // Bounded wait that ignores the abort flag: used while draining in-flight copies or
 // MMAs before the CTA exits, which always complete on their own.
-__device__ __noinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32_t where)
+__device__ __forceinline__ bool drain_wait_inl(uint32_t bar, uint32_t parity, uint32_t where)
 {
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
@@ -66,21 +73,29 @@ __device__ __noinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32_t 
     return true;
 }
 
+__device__ __noinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32_t where)
+{
+    return drain_wait_inl(bar, parity, where);
+}
+
 // Single-thread wait with an inline first probe (the common case: already complete).
+template <bool INL = false>
 __device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, CtaCtl* ctl,
                                           uint32_t where)
 {
-    return mbar_try_wait(bar, parity) || wait_bar(bar, parity, ctl, where);
+    if constexpr (INL) return mbar_try_wait(bar, parity) || wait_bar_inl(bar, parity, ctl, where);
+    else return mbar_try_wait(bar, parity) || wait_bar(bar, parity, ctl, where);
 }
 
 // Warp-wide wait: lane 0 polls (its successful wait is the acquire), the result is
 // broadcast, and a warp barrier -- which orders memory among the lanes, unlike the
 // shuffle -- makes everything lane 0 acquired visible to the other lanes' later loads.
+template <bool INL = false>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, CtaCtl* ctl,
                                           uint32_t where)
 {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = wait_fast(bar, parity, ctl, where) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_fast<INL>(bar, parity, ctl, where) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
@@ -89,12 +104,12 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, CtaCtl*
 // MMA-issue primitives for either a warp-converged issuer (WARP: all 32 lanes call
 // them; each tcgen05 op is executed by one elected lane, which keeps descriptors
 // warp-uniform) or a single issuing thread.
-template <bool WARP>
+template <bool WARP, bool INL = false>
 struct Issuer {
     __device__ static bool wait(uint32_t bar, uint32_t parity, CtaCtl* ctl, uint32_t where)
     {
-        if constexpr (WARP) return warp_wait(bar, parity, ctl, where);
-        else return wait_fast(bar, parity, ctl, where);
+        if constexpr (WARP) return warp_wait<INL>(bar, parity, ctl, where);
+        else return wait_fast<INL>(bar, parity, ctl, where);
     }
     __device__ static void ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc)
     {

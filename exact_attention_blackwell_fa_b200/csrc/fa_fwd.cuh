@@ -76,6 +76,7 @@ struct FwdCfg {
     static constexpr int HALVES = D == 128 ? 1 : 2;
     static constexpr int HALF = 128 / HALVES;    // key columns per softmax warpgroup
     static constexpr int POLY_EVERY = 0;         // exp2 pairs: 1 in POLY_EVERY on the FMA pipe (0: none)
+    static constexpr int POLY_MOD = POLY_EVERY > 0 ? POLY_EVERY : 1;
     static constexpr int UNIT_ROWS = NQ * BM;
     static constexpr uint32_t CHUNK = 32768;
     static constexpr uint32_t QTILE = BM * D * 2;
@@ -249,7 +250,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
                     const int c = cc * 32 + k;
                     const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm2);
                     float e0, e1;
-                    if (C::POLY_EVERY > 0 && !masked && (c >> 1) % C::POLY_EVERY == C::POLY_EVERY - 1) {
+                    if (C::POLY_EVERY > 0 && !masked && (c >> 1) % C::POLY_MOD == C::POLY_MOD - 1) {
                         exp2_fma_x2(x2, e0, e1);
                     } else {
                         const float2 x = f2unpack(x2);
@@ -450,7 +451,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, ui
                         float e0, e1;
                         // one pair in C::POLY_EVERY on the FMA pipe (cubic), the rest on
                         // the SFU; masked tiles use the SFU only (it maps -inf to exactly 0)
-                        if (C::POLY_EVERY > 0 && !masked && (k >> 1) % C::POLY_EVERY == C::POLY_EVERY - 1) {
+                        if (C::POLY_EVERY > 0 && !masked && (k >> 1) % C::POLY_MOD == C::POLY_MOD - 1) {
                             exp2_fma_x2(x2, e0, e1);
                         } else {
                             const float2 x = f2unpack(x2);
