@@ -408,20 +408,7 @@ __device__ void bwd_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, 
             // the whole dQ^T row of this thread's head dim, then TMEM is released (the
             // next dP^T waits for it) before any reduction is issued
             uint32_t r[128];  // r[i] = dQ^T[dim t][query i] of this block
-            {
-                uint32_t (&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
-                uint32_t (&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
-                uint32_t (&a2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
-                uint32_t (&a3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
-                tmem_ld32_nowait(tmem + lane_off + C::T_DP, a0);
-                tmem_ld32_nowait(tmem + lane_off + C::T_DP + 32, a1);
-                tmem_ld32_nowait(tmem + lane_off + C::T_DP + 64, a2);
-                tmem_ld32_nowait(tmem + lane_off + C::T_DP + 96, a3);
-                tmem_wait_ld_dep(a0);
-                tmem_wait_ld_dep(a1);
-                tmem_wait_ld_dep(a2);
-                tmem_wait_ld_dep(a3);
-            }
+            tmem_ld128_split(tmem + lane_off + C::T_DP, r);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));

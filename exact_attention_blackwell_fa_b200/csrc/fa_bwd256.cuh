@@ -7,7 +7,8 @@
 //   * a work unit is 64 keys of one (batch, KV head); it loops over the group's query
 //     heads and 128-row query blocks;
 //   * S = Q K^T and dP = dO V^T are computed query-major (M = 128 query rows, N = 64
-//     keys), so the compute warpgroup's thread owns one query row and its LSE and D;
+//     keys); two compute warpgroups each own 32 of the 64 keys, a thread one query
+//     row (and its LSE and D);
 //   * P and dS go to shared memory as [query][key] tiles (128-byte swizzle); the
 //     key-side accumulators are kept transposed, dV^T += dO^T P and dK^T += Q^T dS,
 //     as two M = 128 head-dim halves each, reading dO, Q (MN-major) and P, dS
@@ -28,8 +29,15 @@ struct Bwd256Cfg {
     static constexpr int D = 256;
     static constexpr int BN = 64;   // keys per unit
     static constexpr int BM = 128;  // query rows per step
-    static constexpr int THREADS = 384;
-    static constexpr int MMA_WARP = 8, LOAD_WARP = 9;
+    // warps 0-7: compute (two warpgroups, 32 keys each), 8-11: dQ, 12: MMA, 13: TMA,
+    // 14-15: idle (they complete the fourth warpgroup for setmaxnreg)
+    static constexpr int THREADS = 512;
+    static constexpr int DQ_WARP = 8, MMA_WARP = 12, LOAD_WARP = 13;
+    // registers per thread: launched at 128; the MMA/TMA warpgroup gives 8 of them to
+    // the dQ warpgroup, which then holds a whole 128-column dQ^T row in registers
+    static constexpr uint32_t REG_LAUNCH = 128, REG_DQ = 136, REG_CTRL = 120;
+    static_assert(8 * 32 * REG_LAUNCH + 4 * 32 * REG_DQ + 4 * 32 * REG_CTRL <= THREADS * REG_LAUNCH,
+                  "register split exceeds the launch budget");
     // lane 0 of the MMA warp issues alone (the converged, elected-lane form measured
     // slower here)
     static constexpr bool WARP_ISSUE = false;
@@ -90,27 +98,30 @@ __device__ __forceinline__ BwdUnit bwd256_decode(const BwdParams& p, int t)
     return u;
 }
 
-// P or dS row of one query (64 keys, 16-bit) into a [128][64] tile, 128-byte swizzle
-__device__ __forceinline__ void store_tile_row(uint32_t tile, int row, const uint32_t (&w)[32])
+// Half of a P or dS row of one query (keys 32h .. 32h+31, 16-bit) into a [128][64]
+// tile, 128-byte swizzle
+__device__ __forceinline__ void store_tile_half_row(uint32_t tile, int row, int half, const uint32_t (&w)[16])
 {
 #pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-        const uint32_t addr = tile + row * 128u + ((static_cast<uint32_t>(c8) ^ (row & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * c8]),
-                     "r"(w[4 * c8 + 1]), "r"(w[4 * c8 + 2]), "r"(w[4 * c8 + 3])
+    for (int c = 0; c < 4; ++c) {
+        const uint32_t c8 = static_cast<uint32_t>(half * 4 + c);
+        const uint32_t addr = tile + row * 128u + ((c8 ^ (row & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * c]),
+                     "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3])
                      : "memory");
     }
 }
 
-// ---- compute warpgroup (thread = query row): P and dS; then the dV / dK epilogue ----
+// ---- compute warpgroups (thread = query row, 32 keys each): P and dS; epilogue ----
 template <bool BF16>
 __device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars,
-                               CtaCtl* ctl, int wq)
+                               CtaCtl* ctl, int wq, int half)
 {
     using C = Bwd256Cfg<BF16>;
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
     const int lane = threadIdx.x & 31;
     const int t = wq * 32 + lane;  // query row within the block, and head-dim lane later
+    const int k0 = half * 32;      // this warpgroup's keys within the unit: k0 .. k0 + 31
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     auto bar = [&](int i) { return bars + 8u * i; };
     const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
@@ -124,75 +135,65 @@ __device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base,
             // key n*64 + c is visible iff c <= lim
             const int lim = i + (p.Sk - p.Sq) - u.n * 64;
             const bool masked = p.causal && (u.n * 64 + 63 > m * 128 + p.Sk - p.Sq);
-            if (!warp_wait(bar(C::B_Q_FULL), it & 1u, ctl, W_B256_Q_FULL)) return;
+            if (!warp_wait<true>(bar(C::B_Q_FULL), it & 1u, ctl, W_B256_Q_FULL)) return;
             float l2, dval;
             asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l2) : "r"(base + C::OFF_ROWS + t * 4u));
             asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dval) : "r"(base + C::OFF_ROWS + 512u + t * 4u));
             const uint64_t negl2 = f2pack(-l2, -l2);
-            if (!warp_wait(bar(C::B_S_FULL), it & 1u, ctl, W_B256_S_FULL)) return;
+            if (!warp_wait<true>(bar(C::B_S_FULL), it & 1u, ctl, W_B256_S_FULL)) return;
             tc_fence_after();
-            uint32_t r0[32], r1[32];
-            tmem_ld32_nowait(tmem + lane_off + C::T_S, r0);
-            tmem_ld32_nowait(tmem + lane_off + C::T_S + 32, r1);
-            tmem_wait_ld_dep(r0);
-            tmem_wait_ld_dep(r1);
-            float P[64];
+            uint32_t r[32];
+            tmem_ld32_wait(tmem + lane_off + C::T_S + k0, r);
+            float P[32];
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-                const uint32_t a = c < 32 ? r0[c] : r1[c - 32];
-                const uint32_t b = c < 32 ? r0[c + 1] : r1[c - 31];
-                const float2 x = f2unpack(ffma2(f2pack(__uint_as_float(a), __uint_as_float(b)), sl2x2, negl2));
-                // all on the SFU (one warp per sub-partition here: nothing hides the
-                // longer FMA-pipe sequence)
+            for (int c = 0; c < 32; c += 2) {
+                const float2 x = f2unpack(ffma2(f2pack(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2x2, negl2));
                 float e0 = ex2_sfu(x.x), e1 = ex2_sfu(x.y);
                 if (masked) {
-                    if (c > lim) e0 = 0.0f;
-                    if (c + 1 > lim) e1 = 0.0f;
+                    if (k0 + c > lim) e0 = 0.0f;
+                    if (k0 + c + 1 > lim) e1 = 0.0f;
                 }
                 P[c] = e0;
                 P[c + 1] = e1;
             }
             {
-                uint32_t w[32];
+                uint32_t w[16];
 #pragma unroll
-                for (int k = 0; k < 32; ++k) w[k] = pack2<BF16>(P[2 * k], P[2 * k + 1]);
-                if (!warp_wait(bar(C::B_P_EMPTY), (it & 1u) ^ 1u, ctl, W_B256_P_EMPTY)) return;
-                store_tile_row(base + C::OFF_P, t, w);
+                for (int k = 0; k < 16; ++k) w[k] = pack2<BF16>(P[2 * k], P[2 * k + 1]);
+                if (!warp_wait<true>(bar(C::B_P_EMPTY), (it & 1u) ^ 1u, ctl, W_B256_P_EMPTY)) return;
+                store_tile_half_row(base + C::OFF_P, t, half, w);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_P_FULL));
 
-            if (!warp_wait(bar(C::B_DP_FULL), it & 1u, ctl, W_B256_DP_FULL)) return;
+            if (!warp_wait<true>(bar(C::B_DP_FULL), it & 1u, ctl, W_B256_DP_FULL)) return;
             tc_fence_after();
-            tmem_ld32_nowait(tmem + lane_off + C::T_DP, r0);
-            tmem_ld32_nowait(tmem + lane_off + C::T_DP + 32, r1);
-            tmem_wait_ld_dep(r0);
-            tmem_wait_ld_dep(r1);
+            tmem_ld32_wait(tmem + lane_off + C::T_DP + k0, r);
             {
-                uint32_t w[32];
+                const uint64_t negd2 = f2pack(-dval, -dval);
+                uint32_t w[16];
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const int c = 2 * k;
-                    const uint32_t a = c < 32 ? r0[c] : r1[c - 32];
-                    const uint32_t b = c < 32 ? r0[c + 1] : r1[c - 31];
-                    w[k] = pack2<BF16>(P[c] * (__uint_as_float(a) - dval), P[c + 1] * (__uint_as_float(b) - dval));
+                for (int k = 0; k < 16; ++k) {
+                    const float2 dd = f2unpack(fadd2(f2pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), negd2));
+                    w[k] = pack2<BF16>(P[2 * k] * dd.x, P[2 * k + 1] * dd.y);
                 }
-                if (!warp_wait(bar(C::B_DS_EMPTY), (it & 1u) ^ 1u, ctl, W_B256_DS_EMPTY)) return;
-                store_tile_row(base + C::OFF_DS, t, w);
+                if (!warp_wait<true>(bar(C::B_DS_EMPTY), (it & 1u) ^ 1u, ctl, W_B256_DS_EMPTY)) return;
+                store_tile_half_row(base + C::OFF_DS, t, half, w);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_DS_FULL));
         }
-        // epilogue: thread t holds head-dim column (half * 128 + t) of dV^T / dK^T
-        if (!warp_wait(bar(C::B_DKV_FINAL), unit_it & 1u, ctl, W_B256_DKV_FINAL)) return;
+        // epilogue: thread t holds head-dim column (hf * 128 + t) of dV^T (half 0) or
+        // dK^T (half 1)
+        if (!warp_wait<true>(bar(C::B_DKV_FINAL), unit_it & 1u, ctl, W_B256_DKV_FINAL)) return;
         ++unit_it;
         tc_fence_after();
-#pragma unroll 1
-        for (int which = 0; which < 2; ++which) {
+        {
+            const int which = half;
             const float mul = which == 0 ? 1.0f : p.scale;
             T* dst = static_cast<T*>(which == 0 ? p.dv : p.dk);
 #pragma unroll 1
@@ -236,18 +237,15 @@ __device__ void bwd256_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bar
             float* blk = p.dqacc + ((static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + m * 128) * C::D + t;
 #pragma unroll 1
             for (int dh = 0; dh < 2; ++dh, ++k) {
-                if (!warp_wait(bar(C::B_DQ_FULL), k & 1u, ctl, W_B256_DQ_FULL)) return;
+                if (!warp_wait<true>(bar(C::B_DQ_FULL), k & 1u, ctl, W_B256_DQ_FULL)) return;
                 tc_fence_after();
                 uint32_t r[128];  // r[i] = dQ^T[dim dh*128 + t][query i]
-                tmem_ld128_wait(tmem + lane_off + C::T_DQ, r);
+                tmem_ld128_split(tmem + lane_off + C::T_DQ, r);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
                 float* dst = blk + dh * 128;
-#pragma unroll
-                for (int i = 0; i < 128; ++i)
-                    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst + i * C::D), "f"(__uint_as_float(r[i]))
-                                 : "memory");
+                red_rows<C::D * 4>(dst, r, std::make_index_sequence<128>{});
             }
         }
     }
@@ -258,7 +256,7 @@ template <bool BF16>
 __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars, CtaCtl* ctl)
 {
     using C = Bwd256Cfg<BF16>;
-    using I = Issuer<C::WARP_ISSUE>;
+    using I = Issuer<C::WARP_ISSUE, true>;
     auto bar = [&](int i) { return bars + 8u * i; };
     const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQ = base + C::OFF_Q,
                    sDO = base + C::OFF_DO, sP = base + C::OFF_P, sDS = base + C::OFF_DS;
@@ -367,7 +365,7 @@ struct Bwd256Load {
         for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
             const BwdUnit u = bwd256_decode(p, ui);
             if (u.T == 0) continue;
-            if (!wait_bar(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_B256_KV_EMPTY)) return;
+            if (!wait_bar_inl(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_B256_KV_EMPTY)) return;
             mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::KV_BYTES);
             for (int blk = 0; blk < 4; ++blk) {
                 tma_load_4d(base + C::OFF_K + blk * C::KV_BLK, tmK, bar(C::B_KV_FULL), blk * 64, u.hkv, u.n * 64, u.b);
@@ -379,7 +377,7 @@ struct Bwd256Load {
                 int h, m;
                 bwd_step(p, u, s, h, m);
                 const uint32_t ph = (it & 1u) ^ 1u;
-                if (!wait_bar(bar(C::B_Q_EMPTY), ph, ctl, W_B256_Q_EMPTY)) return;
+                if (!wait_bar_inl(bar(C::B_Q_EMPTY), ph, ctl, W_B256_Q_EMPTY)) return;
                 mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_BYTES + C::ROWS_BYTES);
                 for (int blk = 0; blk < 4; ++blk)
                     tma_load_4d(base + C::OFF_Q + blk * C::Q_BLK, tmQ, bar(C::B_Q_FULL), blk * 64, h, m * 128, u.b);
@@ -389,7 +387,7 @@ struct Bwd256Load {
                     bulk_load(base + C::OFF_ROWS + 512, p.Dv + rb, 512, bar(C::B_Q_FULL));
                 }
                 q_round = static_cast<int>(it);
-                if (!wait_bar(bar(C::B_DO_EMPTY), ph, ctl, W_B256_DO_EMPTY)) return;
+                if (!wait_bar_inl(bar(C::B_DO_EMPTY), ph, ctl, W_B256_DO_EMPTY)) return;
                 mbar_arrive_expect_tx(bar(C::B_DO_FULL), C::Q_BYTES);
                 for (int blk = 0; blk < 4; ++blk)
                     tma_load_4d(base + C::OFF_DO + blk * C::Q_BLK, tmDO, bar(C::B_DO_FULL), blk * 64, h, m * 128, u.b);
@@ -399,9 +397,9 @@ struct Bwd256Load {
     }
     __device__ void drain()
     {
-        if (kv_round >= 0) drain_wait(bar(C::B_KV_FULL), static_cast<uint32_t>(kv_round) & 1u, W_B256_DRAIN);
-        if (q_round >= 0) drain_wait(bar(C::B_Q_FULL), static_cast<uint32_t>(q_round) & 1u, W_B256_DRAIN);
-        if (do_round >= 0) drain_wait(bar(C::B_DO_FULL), static_cast<uint32_t>(do_round) & 1u, W_B256_DRAIN);
+        if (kv_round >= 0) drain_wait_inl(bar(C::B_KV_FULL), static_cast<uint32_t>(kv_round) & 1u, W_B256_DRAIN);
+        if (q_round >= 0) drain_wait_inl(bar(C::B_Q_FULL), static_cast<uint32_t>(q_round) & 1u, W_B256_DRAIN);
+        if (do_round >= 0) drain_wait_inl(bar(C::B_DO_FULL), static_cast<uint32_t>(do_round) & 1u, W_B256_DRAIN);
     }
 };
 
@@ -427,8 +425,8 @@ __global__ void __launch_bounds__(Bwd256Cfg<BF16>::THREADS, 1)
     if (threadIdx.x == 0) {
         auto bar = [&](int i) { return bars + 8u * i; };
         for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), 1);
-        mbar_init(bar(C::B_P_FULL), 4);
-        mbar_init(bar(C::B_DS_FULL), 4);
+        mbar_init(bar(C::B_P_FULL), 8);
+        mbar_init(bar(C::B_DS_FULL), 8);
         mbar_init(bar(C::B_DQ_EMPTY), 4);
         ctl->abort = 0u;
         fence_mbar_init();
@@ -448,24 +446,30 @@ __global__ void __launch_bounds__(Bwd256Cfg<BF16>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
 
-    if (warp < 4) {
-        bwd256_compute<BF16>(p, tmem, base, bars, ctl, warp);
-    } else if (warp < 8) {
-        bwd256_dq_reduce<BF16>(p, tmem, bars, ctl, warp - 4);
-    } else if (warp == C::MMA_WARP) {
-        if (C::WARP_ISSUE || lane == 0) {
-            bwd256_mma<BF16>(p, tmem, base, bars, ctl);
-            Issuer<C::WARP_ISSUE>::commit(bars + 8u * C::B_DRAIN);
-            if (lane == 0) drain_wait(bars + 8u * C::B_DRAIN, 0u, W_B256_DRAIN);
+    // register split (setmaxnreg, per warpgroup): warps 12-15 release registers on entry
+    // to their branch, unconditionally, so the dQ warpgroup's increase always completes
+    if (warp < C::DQ_WARP) {
+        bwd256_compute<BF16>(p, tmem, base, bars, ctl, warp & 3, warp >> 2);
+    } else if (warp < C::MMA_WARP) {
+        setmaxnreg_inc<C::REG_DQ>();  // completes once warps 12-15 have released theirs
+        bwd256_dq_reduce<BF16>(p, tmem, bars, ctl, warp - C::DQ_WARP);
+    } else {
+        setmaxnreg_dec<C::REG_CTRL>();  // all four warps, first thing, unconditionally
+        if (warp == C::MMA_WARP) {
+            if (C::WARP_ISSUE || lane == 0) {
+                bwd256_mma<BF16>(p, tmem, base, bars, ctl);
+                Issuer<C::WARP_ISSUE, true>::commit(bars + 8u * C::B_DRAIN);
+                if (lane == 0) drain_wait_inl(bars + 8u * C::B_DRAIN, 0u, W_B256_DRAIN);
+            }
+            __syncwarp();
+        } else if (warp == C::LOAD_WARP) {
+            if (lane == 0) {
+                Bwd256Load<BF16> ld{&tmQ, &tmK, &tmV, &tmDO, base, bars, ctl};
+                ld.run(p);
+                ld.drain();
+            }
+            __syncwarp();
         }
-        __syncwarp();
-    } else if (warp == C::LOAD_WARP) {
-        if (lane == 0) {
-            Bwd256Load<BF16> ld{&tmQ, &tmK, &tmV, &tmDO, base, bars, ctl};
-            ld.run(p);
-            ld.drain();
-        }
-        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();

@@ -348,6 +348,25 @@ __device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32])
         : "memory");
 }
 
+// 128 consecutive columns as four 32-column loads in flight, then one wait: the same
+// data as a single .x128 load, usable where the kernel's register target is below
+// what one .x128 instruction needs (code that runs under a raised setmaxnreg budget).
+__device__ __forceinline__ void tmem_ld128_split(uint32_t taddr, uint32_t (&r)[128])
+{
+    uint32_t (&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+    uint32_t (&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+    uint32_t (&a2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
+    uint32_t (&a3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
+    tmem_ld32_nowait(taddr, a0);
+    tmem_ld32_nowait(taddr + 32, a1);
+    tmem_ld32_nowait(taddr + 64, a2);
+    tmem_ld32_nowait(taddr + 96, a3);
+    tmem_wait_ld_dep(a0);
+    tmem_wait_ld_dep(a1);
+    tmem_wait_ld_dep(a2);
+    tmem_wait_ld_dep(a3);
+}
+
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------------
