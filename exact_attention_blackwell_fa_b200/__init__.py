@@ -12,6 +12,7 @@ library's CUDA kernels.  The functions carry the C names:
     fa_last_device_status() -> (code, detail)
     fa_clear_device_status()
     fa_debug_inject(mode)
+    fa_debug_exp2(x, mode=0) -> y
 
 Tensors are CUDA, contiguous, [batch, seq, heads, head_dim], bf16 or fp16; LSE is
 float32 [batch, Hq, Sq].  A non-OK status raises FAError; nothing falls back.
@@ -27,7 +28,7 @@ from . import _lib
 
 __all__ = [
     "FAError", "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
-    "fa_last_device_status", "fa_clear_device_status", "fa_debug_inject",
+    "fa_last_device_status", "fa_clear_device_status", "fa_debug_inject", "fa_debug_exp2",
 ]
 
 
@@ -161,3 +162,14 @@ def fa_clear_device_status(stream=None):
 
 def fa_debug_inject(mode: int):
     _raise(_lib.load().fa_debug_inject(int(mode)), "fa_debug_inject")
+
+
+def fa_debug_exp2(x, mode: int = 0, stream=None):
+    """The kernels' exp2 on a CUDA fp32 tensor: mode 0 the FMA-pipe cubic, 1 the SFU
+    instruction.  Returns a new tensor (enqueued on the stream)."""
+    if x.device.type != "cuda" or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    _raise(_lib.load().fa_debug_exp2(x.data_ptr(), y.data_ptr(), x.numel(), int(mode), _stream_ptr(stream)),
+           "fa_debug_exp2")
+    return y

@@ -180,6 +180,26 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 
 }  // namespace
 
+namespace fa {
+// Test hook kernel: one thread per pair of values, exactly the kernels' exp2 forms.
+__global__ void fa_debug_exp2_kernel(const float* x, float* y, int n, int mode)
+{
+    const int pr = blockIdx.x * blockDim.x + threadIdx.x;
+    const int i0 = 2 * pr, i1 = 2 * pr + 1;
+    if (i0 >= n) return;
+    const float x0 = x[i0], x1 = i1 < n ? x[i1] : x0;
+    float e0, e1;
+    if (mode == 0) {
+        exp2_fma_x2(f2pack(x0, x1), e0, e1);
+    } else {
+        e0 = ex2_sfu(x0);
+        e1 = ex2_sfu(x1);
+    }
+    y[i0] = e0;
+    if (i1 < n) y[i1] = e1;
+}
+}  // namespace fa
+
 extern "C" {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
@@ -327,6 +347,17 @@ fa_status fa_clear_device_status(fa_stream stream)
                                    reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? FA_OK
                : FA_ERR_CUDA;
+}
+
+fa_status fa_debug_exp2(const float* x, float* y, int n, int mode, fa_stream stream)
+{
+    if (n < 0 || (mode != 0 && mode != 1) || (n > 0 && (x == nullptr || y == nullptr))) return FA_ERR_INVALID_ARG;
+    if (n == 0) return FA_OK;
+    const int pairs = (n + 1) / 2;
+    const int threads = 256;
+    const int blocks = (pairs + threads - 1) / threads;
+    fa::fa_debug_exp2_kernel<<<blocks, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n, mode);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status fa_debug_inject(int mode)

@@ -254,8 +254,8 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
             const bool masked = p.causal && (u.n * 128 + 127 > m * 128 + p.Sk - p.Sq);
             const int jlim = j - (p.Sk - p.Sq) - m * 128 - q0;  // visible iff column c >= jlim
             // the Q-tile barrier also covers the staged row terms
-            if (!warp_wait<true>(bar(C::B_Q_FULL + (it & 1)), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
-            if (!warp_wait<true>(bar(C::B_S_FULL), it & 1u, ctl, W_BWD_S_FULL)) return;
+            if (!warp_wait<true, true>(bar(C::B_Q_FULL + (it & 1)), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
+            if (!warp_wait<true, true>(bar(C::B_S_FULL), it & 1u, ctl, W_BWD_S_FULL)) return;
             tc_fence_after();
             // P^T = 2^(S^T scale log2e - LSE log2e), 32 query columns at a time.  The
             // 16-bit P^T words stay in registers for dS: the MMA issues the next S^T into
@@ -301,8 +301,8 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
             if (lane == 0) mbar_arrive(bar(C::B_P_FULL));
 
             // dS^T = P^T (dP^T - D), 32 query columns at a time (next chunk's load in flight)
-            if (!warp_wait<true>(bar(C::B_DP_FULL), it & 1u, ctl, W_BWD_DP_FULL)) return;
-            if (!warp_wait<true>(bar(C::B_DS_EMPTY), (it & 1u) ^ 1u, ctl, W_BWD_DS_EMPTY)) return;
+            if (!warp_wait<true, true>(bar(C::B_DP_FULL), it & 1u, ctl, W_BWD_DP_FULL)) return;
+            if (!warp_wait<true, true>(bar(C::B_DS_EMPTY), (it & 1u) ^ 1u, ctl, W_BWD_DS_EMPTY)) return;
             tc_fence_after();
             tmem_ld32_nowait(tDP, rbuf[0]);
 #pragma unroll
@@ -342,7 +342,7 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
             if (lane == 0) mbar_arrive(bar(C::B_DS_FULL));
         }
         // epilogue: dV and dK rows of this key block
-        if (!warp_wait<true>(bar(C::B_DKV_FINAL), unit_it & 1u, ctl, W_BWD_DKV_FINAL)) return;
+        if (!warp_wait<true, true>(bar(C::B_DKV_FINAL), unit_it & 1u, ctl, W_BWD_DKV_FINAL)) return;
         ++unit_it;
         tc_fence_after();
         const bool row_ok = j < p.Sk;
@@ -403,7 +403,7 @@ __device__ void bwd_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, 
         for (int s = 0; s < u.T; ++s, ++it) {
             int h, m;
             bwd_step(p, u, s, h, m);
-            if (!warp_wait<true>(bar(C::B_DQ_FULL), it & 1u, ctl, W_BWD_DQ_FULL)) return;
+            if (!warp_wait<true, true>(bar(C::B_DQ_FULL), it & 1u, ctl, W_BWD_DQ_FULL)) return;
             tc_fence_after();
             // the whole dQ^T row of this thread's head dim, then TMEM is released (the
             // next dP^T waits for it) before any reduction is issued
@@ -425,7 +425,7 @@ template <bool BF16>
 __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars, CtaCtl* ctl)
 {
     using C = BwdCfg<BF16>;
-    using I = Issuer<C::WARP_ISSUE, true>;
+    using I = Issuer<C::WARP_ISSUE, true, true>;
     auto bar = [&](int i) { return bars + 8u * i; };
     uint32_t it = 0, unit_it = 0, dq_issued = 0;
     // Descriptors are built once; each MMA adds a constant byte offset / 16 to the
@@ -651,7 +651,7 @@ __global__ void __launch_bounds__(BwdCfg<BF16>::THREADS, 1)
         if (warp == C::MMA_WARP) {
             if (C::WARP_ISSUE || lane == 0) {
                 bwd_mma<BF16>(p, tmem, base, bars, ctl);
-                Issuer<C::WARP_ISSUE, true>::commit(bars + 8u * C::B_DRAIN);
+                Issuer<C::WARP_ISSUE, true, true>::commit(bars + 8u * C::B_DRAIN);
                 if (lane == 0) drain_wait_inl(bars + 8u * C::B_DRAIN, 0u, W_BWD_DRAIN);
             }
             __syncwarp();

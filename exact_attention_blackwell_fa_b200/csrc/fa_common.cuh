@@ -13,6 +13,12 @@ namespace fa {
 
 // Every wait in the kernels gives up after this long and reports FA_ERR_DEVICE_TIMEOUT.
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;
+// Spinning waits (SPIN below) first poll without suspending (test_wait) for this many
+// probes, then fall back to the suspending, timed loop: a thread suspended in try_wait
+// was measured to resume hundreds of cycles after the phase completed, which costs a
+// pipeline whose step time is made of such hand-offs; the polls in turn take issue
+// slots from the warps they share a scheduler with, so each kernel chooses.
+constexpr uint32_t kSpinPolls = 1u << 16;
 
 // Device status: [0] fa_status code of the first failure, [1] code of the wait that
 // gave up, [2] block index, [3] unused.
@@ -78,24 +84,31 @@ __device__ __noinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32_t 
     return drain_wait_inl(bar, parity, where);
 }
 
-// Single-thread wait with an inline first probe (the common case: already complete).
-template <bool INL = false>
+// Single-thread wait: one inline probe (SPIN: a bounded non-suspending poll), then the
+// timed wait.
+template <bool INL = false, bool SPIN = false>
 __device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, CtaCtl* ctl,
                                           uint32_t where)
 {
-    if constexpr (INL) return mbar_try_wait(bar, parity) || wait_bar_inl(bar, parity, ctl, where);
-    else return mbar_try_wait(bar, parity) || wait_bar(bar, parity, ctl, where);
+    if constexpr (SPIN) {
+        for (uint32_t i = 0; i < kSpinPolls; ++i)
+            if (mbar_test_wait(bar, parity)) return true;
+    } else {
+        if (mbar_try_wait(bar, parity)) return true;
+    }
+    if constexpr (INL) return wait_bar_inl(bar, parity, ctl, where);
+    else return wait_bar(bar, parity, ctl, where);
 }
 
 // Warp-wide wait: lane 0 polls (its successful wait is the acquire), the result is
 // broadcast, and a warp barrier -- which orders memory among the lanes, unlike the
 // shuffle -- makes everything lane 0 acquired visible to the other lanes' later loads.
-template <bool INL = false>
+template <bool INL = false, bool SPIN = false>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, CtaCtl* ctl,
                                           uint32_t where)
 {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = wait_fast<INL>(bar, parity, ctl, where) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_fast<INL, SPIN>(bar, parity, ctl, where) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
@@ -104,12 +117,12 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, CtaCtl*
 // MMA-issue primitives for either a warp-converged issuer (WARP: all 32 lanes call
 // them; each tcgen05 op is executed by one elected lane, which keeps descriptors
 // warp-uniform) or a single issuing thread.
-template <bool WARP, bool INL = false>
+template <bool WARP, bool INL = false, bool SPIN = false>
 struct Issuer {
     __device__ static bool wait(uint32_t bar, uint32_t parity, CtaCtl* ctl, uint32_t where)
     {
-        if constexpr (WARP) return warp_wait<INL>(bar, parity, ctl, where);
-        else return wait_fast<INL>(bar, parity, ctl, where);
+        if constexpr (WARP) return warp_wait<INL, SPIN>(bar, parity, ctl, where);
+        else return wait_fast<INL, SPIN>(bar, parity, ctl, where);
     }
     __device__ static void ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc)
     {

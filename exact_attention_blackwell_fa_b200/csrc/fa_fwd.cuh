@@ -199,7 +199,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
         float m_ref = -INFINITY;  // running reference max (log2 units)
         float l = 0.0f;           // running row sum against m_ref
         for (int j = 0; j < n; ++j, ++s_it) {
-            if (!warp_wait(bar(C::B_S_FULL + q), s_it & 1u, ctl, W_FWD_S_FULL)) return;
+            if (!warp_wait<false, true>(bar(C::B_S_FULL + q), s_it & 1u, ctl, W_FWD_S_FULL)) return;
             tc_fence_after();
             uint32_t sr[128];
             {
@@ -282,7 +282,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
             if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q));
         }
         // epilogue: wait for the unit's last P V, normalise and store O and LSE
-        if (!warp_wait(bar(C::B_O_FINAL + q), tile_it & 1u, ctl, W_FWD_O_FINAL)) return;
+        if (!warp_wait<false, true>(bar(C::B_O_FINAL + q), tile_it & 1u, ctl, W_FWD_O_FINAL)) return;
         ++tile_it;
         tc_fence_after();
         const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
@@ -543,7 +543,8 @@ template <int D, bool BF16>
 struct FwdMma {
     using C = FwdCfg<D, BF16>;
     static constexpr bool WARP_ISSUE = D == 256;
-    using I = Issuer<WARP_ISSUE>;
+    static constexpr bool SPIN = D == 128;  // spinning waits measured faster at d=128 only
+    using I = Issuer<WARP_ISSUE, false, SPIN>;
     uint32_t tmem, sQ, sRing, bars;
     CtaCtl* ctl;
     uint32_t seq = 0;  // ring chunk sequence number

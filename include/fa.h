@@ -136,6 +136,17 @@ fa_status fa_clear_device_status(fa_stream stream);
  */
 fa_status fa_debug_inject(int mode);
 
+/*
+ * Test hook: evaluates the kernels' base-2 exponential on `n` fp32 values.
+ * `x` and `y` are device pointers to n floats (caller-owned; y may not alias x).
+ * mode 0: the FMA-pipe cubic of the exp2 split ("Software-exponentials via
+ * CUDA-kernen", FlashAttention 4 page: 2^x = 2^n * p(f), p our relative-minimax
+ * cubic; inputs below -126 are clamped there); mode 1: the SFU instruction
+ * (ex2.approx.ftz).  Enqueued on `stream`, not synchronised.  FA_ERR_INVALID_ARG
+ * for n < 0, an unknown mode, or a null pointer with n > 0.
+ */
+fa_status fa_debug_exp2(const float* x, float* y, int n, int mode, fa_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
