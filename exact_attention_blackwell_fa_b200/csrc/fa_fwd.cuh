@@ -11,26 +11,24 @@
 //     (batch, query head, block of query rows); units are grouped by heads so that the
 //     CTAs running at the same time share K/V through L2, and for the causal mask the
 //     longest units (last query blocks) go first;
-//   * one TMA warp stages Q once per unit and streams K and V through a 4-deep ring
+//   * one TMA warp stages Q once per unit and streams K and V through a 5-deep ring
 //     of 32-KB shared-memory chunks (128 rows x 128 head-dim columns, 128-byte
 //     swizzle) guarded by full/empty mbarriers;
-//   * one thread issues tcgen05.mma: S = Q K^T into TMEM, then O += P V with P read
+//   * one MMA warp issues tcgen05.mma: S = Q K^T into TMEM, then O += P V with P read
 //     back from TMEM (P overwrites the first half of its own S buffer as 16-bit
 //     pairs);
-//   * softmax warpgroups (thread = query row) load S from TMEM, apply the scale and
+//   * one softmax warpgroup per Q tile (thread = one query row holding all 128 key
+//     columns of a tile in registers) loads S from TMEM, applies the scale and
 //     mask, keep the running row max and sum, rescale O in TMEM only when the row max
 //     grew by more than kRescaleTau (log2 units), write P back into TMEM as 16-bit
 //     pairs, and finally normalise and write O and LSE.  The exp2 can be split
 //     between the SFU and an FMA-pipe cubic (FwdCfg::POLY_EVERY); on sm_100 the SFU
 //     alone measured faster for both head dims, so the split is off;
 //
-// head_dim 128: two Q tiles (256 query rows) per unit, TMEM = S0 | S1 | O0 | O1, one
-// softmax warpgroup per Q tile holding a whole 128-key row in registers; the tensor
-// core alternates between the two tiles so that one tile's softmax overlaps the
-// other tile's MMAs.  head_dim 256: one Q tile, TMEM = S(a) | S(b) | O (256
-// columns), S double buffered so the next S = Q K^T runs during the softmax; two
-// softmax warpgroups each own 64 of the 128 key columns and swap half-row maxima
-// through shared memory (speculatively: see fwd_softmax).
+// head_dim 128: two Q tiles (256 query rows) per unit, TMEM = S0 | S1 | O0 | O1; the
+// tensor core alternates between the two tiles so that one tile's softmax overlaps
+// the other tile's MMAs.  head_dim 256: one Q tile, TMEM = S(a) | S(b) | O (256
+// columns), S double buffered so the next S = Q K^T runs during the softmax.
 #pragma once
 
 #include <type_traits>
@@ -58,7 +56,7 @@ struct FwdParams {
 // wait-site codes reported through the device status word
 enum : uint32_t {
     W_FWD_Q_FULL = 0x101, W_FWD_Q_EMPTY, W_FWD_RING_FULL, W_FWD_RING_EMPTY, W_FWD_S_FULL,
-    W_FWD_P_FULL, W_FWD_O_DONE, W_FWD_O_FINAL, W_FWD_DRAIN, W_FWD_XMAX, W_FWD_XSUM,
+    W_FWD_P_FULL, W_FWD_O_DONE, W_FWD_O_FINAL, W_FWD_DRAIN, W_FWD_RESERVED_A, W_FWD_RESERVED_B,
     W_FWD_SMEM_ALIGN
 };
 
@@ -68,20 +66,18 @@ struct FwdCfg {
     static constexpr int NQ = D == 128 ? 2 : 1;  // 128-row Q tiles per work unit
     static constexpr int NS = D == 128 ? 1 : 2;  // S buffers per Q tile
     static constexpr int KCH = D / 128;          // 32-KB chunks per K (or V) tile
-    static constexpr int NSTAGE = 4;             // ring depth, in chunks
+    static constexpr int NSTAGE = 5;             // ring depth, in chunks
     static constexpr int BM = 128;               // query rows per Q tile
     static constexpr int BN = 128;               // keys per KV tile
-    // softmax warpgroups per Q tile: head_dim 128 uses one (thread = a whole 128-key
-    // row); head_dim 256 two, each owning 64 of the 128 key columns
-    static constexpr int HALVES = D == 128 ? 1 : 2;
-    static constexpr int HALF = 128 / HALVES;    // key columns per softmax warpgroup
     static constexpr int POLY_EVERY = 0;         // exp2 pairs: 1 in POLY_EVERY on the FMA pipe (0: none)
     static constexpr int POLY_MOD = POLY_EVERY > 0 ? POLY_EVERY : 1;
+    // spinning waits (see fa_common.cuh) for the softmax and MMA warps
+    static constexpr bool SPIN = D == 128;
     static constexpr int UNIT_ROWS = NQ * BM;
     static constexpr uint32_t CHUNK = 32768;
     static constexpr uint32_t QTILE = BM * D * 2;
     static constexpr uint32_t Q_BYTES = NQ * QTILE;
-    static constexpr int SOFTMAX_WARPS = NQ * HALVES * 4;
+    static constexpr int SOFTMAX_WARPS = NQ * 4;     // one warpgroup per Q tile
     static constexpr int CTRL_WARP = SOFTMAX_WARPS;  // MMA warp; the TMA warp follows it
     static constexpr int THREADS = (SOFTMAX_WARPS + 2) * 32;
 
@@ -89,9 +85,7 @@ struct FwdCfg {
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_RING = Q_BYTES;
     // half-row maxima, [Q tile][step parity][half][row], then half-row sums [Q tile][half][row]
-    static constexpr uint32_t OFF_XMAX = OFF_RING + NSTAGE * CHUNK;
-    static constexpr uint32_t OFF_XSUM = OFF_XMAX + NQ * 2 * 2 * BM * 4;
-    static constexpr uint32_t OFF_BAR = OFF_XSUM + NQ * 2 * BM * 4;
+    static constexpr uint32_t OFF_BAR = OFF_RING + NSTAGE * CHUNK;
     // barrier indices
     static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1;
     static constexpr int B_FULL = 2;
@@ -100,9 +94,7 @@ struct FwdCfg {
     static constexpr int B_P_FULL = B_S_FULL + NQ * NS;
     static constexpr int B_O_DONE = B_P_FULL + NQ * NS;
     static constexpr int B_O_FINAL = B_O_DONE + NQ;
-    static constexpr int B_XMAX = B_O_FINAL + NQ;  // [Q tile][step parity]
-    static constexpr int B_XSUM = B_XMAX + 2 * NQ;
-    static constexpr int B_DRAIN = B_XSUM + NQ;
+    static constexpr int B_DRAIN = B_O_FINAL + NQ;
     static constexpr int NBAR = B_DRAIN + 1;
     static constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
     // no alignment slack: the kernel checks that the base is 1024-byte aligned
@@ -112,14 +104,9 @@ struct FwdCfg {
     // TMEM columns
     __device__ static constexpr uint32_t col_S(int q, int sb) { return NQ == 2 ? q * 128 : sb * 128; }
     __device__ static constexpr uint32_t col_O(int q) { return 256 + q * 128; }
-    // P for key columns 64h .. 64h+63 is written by softmax half h over the first 32
-    // columns of its own (already consumed) half of the S buffer
-    __device__ static constexpr uint32_t col_P(int half) { return half * 64; }
-    // TMEM column of the packed P words for keys 16 kk .. 16 kk + 15
-    __device__ static constexpr uint32_t col_Pk(int kk)
-    {
-        return HALVES == 2 ? col_P(kk >> 2) + (kk & 3) * 8 : kk * 8;
-    }
+    // P is written over the first 64 columns of its (consumed) S buffer as 16-bit
+    // pairs: the packed words for keys 16 kk .. 16 kk + 15 sit at column 8 kk
+    __device__ static constexpr uint32_t col_Pk(int kk) { return kk * 8; }
 
     static constexpr uint32_t IDESC_S = idesc_f16(BF16, 128, 128, false, false);
     static constexpr uint32_t IDESC_PV = idesc_f16(BF16, 128, 128, false, true);
@@ -155,19 +142,17 @@ __device__ __forceinline__ int fwd_kv_tiles(const FwdParams& p, int m0)
 }
 
 // ---------------------------------------------------------------------------------
-// Softmax / epilogue warpgroup, one per 128-row Q tile (head_dim 128): thread = one
-// query row, all 128 key columns of a tile held in registers.
+// Softmax / epilogue warpgroup, one per 128-row Q tile: thread = one query row, all
+// 128 key columns of a tile held in registers.
 // ---------------------------------------------------------------------------------
 template <int D, bool BF16>
 __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int q, int wq)
 {
     using C = FwdCfg<D, BF16>;
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-    static_assert(C::HALVES == 1 && C::NS == 1, "row softmax: one warpgroup, one S buffer per Q tile");
     const int lane = threadIdx.x & 31;
     const int r_in_tile = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::col_S(q, 0);
     const uint32_t tO = tmem + lane_off + C::col_O(q);
     auto bar = [&](int i) { return bars + 8u * i; };
     const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
@@ -199,7 +184,10 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
         float m_ref = -INFINITY;  // running reference max (log2 units)
         float l = 0.0f;           // running row sum against m_ref
         for (int j = 0; j < n; ++j, ++s_it) {
-            if (!warp_wait<false, true>(bar(C::B_S_FULL + q), s_it & 1u, ctl, W_FWD_S_FULL)) return;
+            const int sb = s_it % C::NS;
+            const uint32_t tS = tmem + lane_off + C::col_S(q, sb);
+            if (!warp_wait<false, C::SPIN>(bar(C::B_S_FULL + q * C::NS + sb), (s_it / C::NS) & 1u, ctl, W_FWD_S_FULL))
+                return;
             tc_fence_after();
             uint32_t sr[128];
             {
@@ -263,9 +251,15 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
                 tmem_st16(tS + cc * 16, pk);
             }
             const float2 a = f2unpack(fadd2(acc2[0], acc2[1]));
-            // O holds every earlier P V product here (S_full of this tile was committed
-            // after the previous P V), so it can be rescaled before this P is released
+            // O must hold every earlier P V product before it is rescaled: with one S
+            // buffer S_full of this tile was committed after the previous P V; with two,
+            // wait for the previous P V (the MMA commits O_done after each one)
             if (__any_sync(0xffffffffu, resc)) {
+                if (C::NS == 2) {
+                    if (!warp_wait<false, C::SPIN>(bar(C::B_O_DONE + q), (s_it - 1u) & 1u, ctl, W_FWD_O_DONE))
+                        return;
+                    tc_fence_after();
+                }
 #pragma unroll 1
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t r[32];
@@ -279,10 +273,10 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q));
+            if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q * C::NS + sb));
         }
         // epilogue: wait for the unit's last P V, normalise and store O and LSE
-        if (!warp_wait<false, true>(bar(C::B_O_FINAL + q), tile_it & 1u, ctl, W_FWD_O_FINAL)) return;
+        if (!warp_wait<false, C::SPIN>(bar(C::B_O_FINAL + q), tile_it & 1u, ctl, W_FWD_O_FINAL)) return;
         ++tile_it;
         tc_fence_after();
         const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
@@ -308,232 +302,6 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
 }
 
 // ---------------------------------------------------------------------------------
-// Softmax / epilogue warpgroups: two per Q tile, `half` owns key columns 64h..64h+63.
-// ---------------------------------------------------------------------------------
-template <int D, bool BF16>
-__device__ void fwd_softmax(const FwdParams& p, uint32_t tmem, uint32_t bars, uint8_t* smem,
-                            CtaCtl* ctl, int q, int half, int wq)
-{
-    using C = FwdCfg<D, BF16>;
-    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-    constexpr int OCOLS = D / 2;  // O columns this warpgroup rescales and stores
-    const int lane = threadIdx.x & 31;
-    const int r_in_tile = wq * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tO = tmem + lane_off + C::col_O(q) + half * OCOLS;
-    float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX) + q * (2 * 2 * C::BM);
-    float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM) + q * (2 * C::BM);
-    auto bar = [&](int i) { return bars + 8u * i; };
-    const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
-    uint32_t s_it = 0, pv_it = 0, tile_it = 0;
-
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-        int b, h, m0;
-        fwd_decode<C::UNIT_ROWS>(p, t, b, h, m0);
-        const int n = fwd_kv_tiles<C::UNIT_ROWS>(p, m0);
-        const int q0 = m0 + q * C::BM;  // first query row of this Q tile
-        const int row = q0 + r_in_tile;
-        const bool row_ok = row < p.Sq;
-        T* orow = reinterpret_cast<T*>(p.o) + ((static_cast<size_t>(b) * p.Sq + row) * p.Hq + h) * D +
-                  half * OCOLS;
-        float* lrow = p.lse + (static_cast<size_t>(b) * p.Hq + h) * p.Sq + row;
-        if (n == 0) {  // causal with Sq > Sk: no key is visible to any row of the unit
-            if (row_ok) {
-                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                for (int c = 0; c < OCOLS / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
-                if (half == 0) *lrow = -INFINITY;
-            }
-            continue;
-        }
-        // columns >= lim are masked for this row; the tile-level test uses the first
-        // row of the Q tile, which has the smallest limit
-        const int lim = p.causal ? min(p.Sk, row + p.Sk - p.Sq + 1) : p.Sk;
-        const int lim0 = p.causal ? min(p.Sk, q0 + p.Sk - p.Sq + 1) : p.Sk;
-
-        float m_ref = -INFINITY;  // running reference max (log2 units), same in both halves
-        float l = 0.0f;           // running sum of this half's columns against m_ref
-        for (int j = 0; j < n; ++j) {
-            const int sb = s_it % C::NS;
-            if (!warp_wait(bar(C::B_S_FULL + q * C::NS + sb), (s_it / C::NS) & 1u, ctl, W_FWD_S_FULL))
-                return;
-            tc_fence_after();
-            const uint32_t tS = tmem + lane_off + C::col_S(q, sb) + half * C::HALF;
-            uint32_t r0[32], r1[32];
-            tmem_ld32_nowait(tS, r0);
-            tmem_ld32_nowait(tS + 32, r1);
-            tmem_wait_ld_dep(r0);
-            tmem_wait_ld_dep(r1);
-            const int c0 = j * C::BN + half * C::HALF;  // key index of column 0 of this half
-            const bool masked = c0 + C::HALF > lim0;
-            if (masked) {
-                const int cut = lim - c0;
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    if (c >= cut) r0[c] = __float_as_uint(-INFINITY);
-                    if (c + 32 >= cut) r1[c] = __float_as_uint(-INFINITY);
-                }
-            }
-            float mx[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) mx[i] = fmaxf(__uint_as_float(r0[i]), __uint_as_float(r1[i]));
-#pragma unroll
-            for (int c = 4; c < 32; c += 4)
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    mx[i] = fmax3(mx[i], __uint_as_float(r0[c + i]), __uint_as_float(r1[c + i]));
-            const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            // publish this half-row maximum to the other warpgroup of the Q tile
-            const int par = s_it & 1;
-            xmax[(par * 2 + half) * C::BM + r_in_tile] = hmax;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_XMAX + q * 2 + par));
-
-            // Reference update for the whole row: both halves see the same two maxima and
-            // reach the same decision.
-            auto update_reference = [&](float partner) -> bool {
-                const float m_tile = fmaxf(hmax, partner) * p.sl2;  // scale > 0
-                const float m_new = fmaxf(m_ref, m_tile);
-                const bool resc = (m_ref != -INFINITY) && (m_new - m_ref > kRescaleTau);
-                if (m_ref == -INFINITY) m_ref = m_new;
-                if (__any_sync(0xffffffffu, resc)) {
-                    // O must hold every earlier P V product before it is scaled: with one
-                    // S buffer that is implied by S_full (the MMA issued S after the
-                    // previous P V); with two, wait for the previous P V explicitly.
-                    if (C::NS == 2) {
-                        if (!warp_wait(bar(C::B_O_DONE + q), (pv_it - 1u) & 1u, ctl, W_FWD_O_DONE))
-                            return false;
-                        tc_fence_after();
-                    }
-                    const float alpha = resc ? ex2_sfu(m_ref - m_new) : 1.0f;
-#pragma unroll 1
-                    for (int cc = 0; cc < OCOLS / 32; ++cc) {
-                        uint32_t r[32];
-                        tmem_ld32_wait(tO + cc * 32, r);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-                        tmem_st32(tO + cc * 32, r);
-                    }
-                    tmem_wait_st();
-                    if (resc) {
-                        l *= alpha;
-                        m_ref = m_new;
-                    }
-                }
-                return true;
-            };
-            const uint32_t tP = tmem + lane_off + C::col_S(q, sb) + C::col_P(half);
-            // P = 2^(S scale log2e - m_ref) for this half, into registers: the S values are
-            // loaded again, 32 columns at a time (the second load in flight while the first
-            // is used), which keeps the register footprint small.  S stays intact in TMEM
-            // until store_p, so the pass can be redone.
-            uint32_t pk[32];
-            auto exp_pass = [&]() -> float {
-                const float negm = (m_ref == -INFINITY) ? 0.0f : -m_ref;
-                const uint64_t negm2 = f2pack(negm, negm);
-                uint64_t acc2[2] = {f2pack(0.0f, 0.0f), f2pack(0.0f, 0.0f)};
-                tmem_ld32_nowait(tS, r0);
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    uint32_t (&r)[32] = cc == 0 ? r0 : r1;
-                    tmem_wait_ld_dep(r);
-                    if (cc == 0) tmem_ld32_nowait(tS + 32, r1);
-                    if (masked) {
-                        const int cut = lim - c0 - cc * 32;
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (c >= cut) r[c] = __float_as_uint(-INFINITY);
-                    }
-#pragma unroll
-                    for (int k = 0; k < 32; k += 2) {
-                        const uint64_t x2 =
-                            ffma2(f2pack(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), sl2x2, negm2);
-                        float e0, e1;
-                        // one pair in C::POLY_EVERY on the FMA pipe (cubic), the rest on
-                        // the SFU; masked tiles use the SFU only (it maps -inf to exactly 0)
-                        if (C::POLY_EVERY > 0 && !masked && (k >> 1) % C::POLY_MOD == C::POLY_MOD - 1) {
-                            exp2_fma_x2(x2, e0, e1);
-                        } else {
-                            const float2 x = f2unpack(x2);
-                            e0 = ex2_sfu(x.x);
-                            e1 = ex2_sfu(x.y);
-                        }
-                        acc2[(k >> 1) & 1] = fadd2(acc2[(k >> 1) & 1], f2pack(e0, e1));
-                        pk[cc * 16 + (k >> 1)] = pack2_p<BF16>(e0, e1);
-                    }
-                }
-                const float2 a = f2unpack(fadd2(acc2[0], acc2[1]));
-                return a.x + a.y;
-            };
-            // P overwrites the first 32 columns of this half's (consumed) S columns
-            auto store_p = [&]() {
-                const uint32_t tP = tmem + lane_off + C::col_S(q, sb) + C::col_P(half);
-                tmem_st16(tP, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-                tmem_st16(tP + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
-                tmem_wait_st();
-            };
-            const float m_loc = hmax * p.sl2;
-            // With an established reference and this half's maximum within kRescaleTau of it
-            // (the common case after the first tile), P is computed before the other half's
-            // maximum is known; if that maximum then forces a new reference, the pass is
-            // redone.  Otherwise the maxima are swapped first.
-            const bool speculate =
-                !__any_sync(0xffffffffu, m_ref == -INFINITY || m_loc - m_ref > kRescaleTau);
-            float tile_sum;
-            if (speculate) {
-                tile_sum = exp_pass();
-                if (!warp_wait(bar(C::B_XMAX + q * 2 + par), (s_it >> 1) & 1u, ctl, W_FWD_XMAX)) return;
-                const float partner = xmax[(par * 2 + (half ^ 1)) * C::BM + r_in_tile];
-                const float m_before = m_ref;
-                if (!update_reference(partner)) return;
-                if (__any_sync(0xffffffffu, m_ref != m_before)) tile_sum = exp_pass();
-            } else {
-                if (!warp_wait(bar(C::B_XMAX + q * 2 + par), (s_it >> 1) & 1u, ctl, W_FWD_XMAX)) return;
-                if (!update_reference(xmax[(par * 2 + (half ^ 1)) * C::BM + r_in_tile])) return;
-                tile_sum = exp_pass();
-            }
-            store_p();
-            l += tile_sum;
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q * C::NS + sb));
-            ++s_it;
-            ++pv_it;
-        }
-        // epilogue: combine the halves' row sums, wait for the unit's last P V,
-        // normalise and store this half of O (and LSE, from half 0)
-        xsum[half * C::BM + r_in_tile] = l;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::B_XSUM + q));
-        if (!warp_wait(bar(C::B_XSUM + q), tile_it & 1u, ctl, W_FWD_XSUM)) return;
-        const float l_all = l + xsum[(half ^ 1) * C::BM + r_in_tile];
-        if (!warp_wait(bar(C::B_O_FINAL + q), tile_it & 1u, ctl, W_FWD_O_FINAL)) return;
-        ++tile_it;
-        tc_fence_after();
-        const float inv = (l_all > 0.0f) ? 1.0f / l_all : 0.0f;
-#pragma unroll 1
-        for (int cc = 0; cc < OCOLS / 32; ++cc) {
-            uint32_t r[32];
-            tmem_ld32_wait(tO + cc * 32, r);
-            uint32_t pk[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                pk[k] = pack2<BF16>(__uint_as_float(r[2 * k]) * inv, __uint_as_float(r[2 * k + 1]) * inv);
-            if (row_ok) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
-                dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
-            }
-        }
-        if (row_ok && half == 0)
-            *lrow = (l_all > 0.0f) ? (m_ref + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
-        tc_fence_before();
-    }
-}
-
-// ---------------------------------------------------------------------------------
 // MMA issuer.  head_dim 256: the whole warp runs the issue loop, converged, and each
 // tcgen05 op is executed by one elected lane (warp-uniform descriptors, few
 // instructions per MMA).  head_dim 128: lane 0 alone runs it (the converged form
@@ -543,8 +311,7 @@ template <int D, bool BF16>
 struct FwdMma {
     using C = FwdCfg<D, BF16>;
     static constexpr bool WARP_ISSUE = D == 256;
-    static constexpr bool SPIN = D == 128;  // spinning waits measured faster at d=128 only
-    using I = Issuer<WARP_ISSUE, false, SPIN>;
+    using I = Issuer<WARP_ISSUE, false, C::SPIN>;
     uint32_t tmem, sQ, sRing, bars;
     CtaCtl* ctl;
     uint32_t seq = 0;  // ring chunk sequence number
@@ -840,14 +607,11 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
         }
         for (int i = 0; i < C::NQ * C::NS; ++i) {
             mbar_init(bar(C::B_S_FULL + i), 1);
-            mbar_init(bar(C::B_P_FULL + i), 4 * C::HALVES);  // one arrive per softmax warp of the tile
+            mbar_init(bar(C::B_P_FULL + i), 4);  // one arrive per softmax warp of the tile
         }
         for (int q = 0; q < C::NQ; ++q) {
             mbar_init(bar(C::B_O_DONE + q), 1);
             mbar_init(bar(C::B_O_FINAL + q), 1);
-            mbar_init(bar(C::B_XMAX + 2 * q), 8);
-            mbar_init(bar(C::B_XMAX + 2 * q + 1), 8);
-            mbar_init(bar(C::B_XSUM + q), 8);
         }
         mbar_init(bar(C::B_DRAIN), 1);
         ctl->abort = 0u;
@@ -868,10 +632,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
     const uint32_t tmem = ctl->tmem_base;
 
     if (warp < C::SOFTMAX_WARPS) {
-        if constexpr (C::HALVES == 1)
-            fwd_softmax_row<D, BF16>(p, tmem, bars, ctl, warp >> 2, warp & 3);
-        else
-            fwd_softmax<D, BF16>(p, tmem, bars, smem_raw, ctl, warp >> 3, (warp >> 2) & 1, warp & 3);
+        fwd_softmax_row<D, BF16>(p, tmem, bars, ctl, warp / 4, warp & 3);
     } else if (warp == C::CTRL_WARP) {
         using M = FwdMma<D, BF16>;
         if (M::WARP_ISSUE || lane == 0) {
