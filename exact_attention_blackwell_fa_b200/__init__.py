@@ -5,6 +5,8 @@ device memory and the current stream; every step of the computation runs in the
 library's CUDA kernels.  The functions carry the C names:
 
     fa_fwd(q, k, v, causal=False, scale=None) -> (o, lse)
+    fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                  seqused_k=None, causal=False, scale=None) -> (o, lse)
     fa_bwd(q, k, v, o, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
     fa_bwd_workspace_size(B, Sq, Hq, d) -> int
     fa_bwd_noalloc(q, k, v, o, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
@@ -27,7 +29,7 @@ import torch
 from . import _lib
 
 __all__ = [
-    "FAError", "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
+    "FAError", "fa_fwd", "fa_fwd_varlen", "fa_bwd", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
     "fa_last_device_status", "fa_clear_device_status", "fa_debug_inject", "fa_debug_exp2",
 ]
 
@@ -92,6 +94,43 @@ def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, 
                               lse.data_ptr(), B, Sq, Sk, Hq, Hkv, d, int(bool(causal)),
                               float(scale), _dtype_code(q), _stream_ptr(stream))
     _raise(code, "fa_fwd")
+    return out, lse
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                  seqused_k=None, causal: bool = False, scale: float | None = None, out=None, lse=None,
+                  stream=None):
+    """Forward over packed variable-length sequences.  q [total_q,Hq,d], k/v
+    [total_k,Hkv,d], cu_seqlens_* int32 CUDA [B+1], seqused_k int32 CUDA [B] or None
+    -> (o [total_q,Hq,d], lse [Hq,total_q] fp32)."""
+    _check(q, "q")
+    _check(k, "k", q.dtype)
+    _check(v, "v", q.dtype)
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    if k.shape != v.shape or k.shape[2] != d:
+        raise ValueError("fa: k and v must be [total_k, Hkv, d] matching q")
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)) + (
+            (("seqused_k", seqused_k),) if seqused_k is not None else ()):
+        if t.device.type != "cuda" or t.dtype != torch.int32 or not t.is_contiguous():
+            raise ValueError(f"fa: {name} must be a contiguous CUDA int32 tensor")
+    B = cu_seqlens_q.numel() - 1
+    if B < 1 or cu_seqlens_k.numel() != B + 1 or (seqused_k is not None and seqused_k.numel() != B):
+        raise ValueError("fa: cu_seqlens_q / cu_seqlens_k need B+1 entries, seqused_k B")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(Hq, total_q, dtype=torch.float32, device=q.device)
+    _check(out, "out", q.dtype)
+    _check(lse, "lse", torch.float32)
+    code = _lib.load().fa_fwd_varlen(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), cu_seqlens_q.data_ptr(),
+        cu_seqlens_k.data_ptr(), seqused_k.data_ptr() if seqused_k is not None else None, B,
+        int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, Hq, Hkv, d, int(bool(causal)),
+        float(scale), _dtype_code(q), _stream_ptr(stream))
+    _raise(code, "fa_fwd_varlen")
     return out, lse
 
 

@@ -222,6 +222,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     fa::FwdParams p{};
     p.o = o;
     p.lse = lse;
+    p.Sq_alloc = Sq;
     p.B = B;
     p.Sq = Sq;
     p.Sk = Sk;
@@ -232,6 +233,57 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     p.num_m = (Sq + unit - 1) / unit;
     p.num_tiles = B * Hq * p.num_m;
     p.chunk_heads = chunk_heads_for(B, Hq, p.group, Sk, d);
+    p.causal = causal ? 1 : 0;
+    p.inject = take_inject();
+    p.sl2 = scale * 1.4426950408889634f;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128)
+        return bf16 ? launch_fwd<128, true>(tq, tk, tv, p, di.sm_count, s)
+                    : launch_fwd<128, false>(tq, tk, tv, p, di.sm_count, s);
+    return bf16 ? launch_fwd<256, true>(tq, tk, tv, p, di.sm_count, s)
+                : launch_fwd<256, false>(tq, tk, tv, p, di.sm_count, s);
+}
+
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, const int* seqused_k, int B,
+                        int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv,
+                        int d, int causal, float scale, fa_dtype dt, fa_stream stream)
+{
+    if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
+    if (total_q < 1 || total_k < 1) return FA_ERR_INVALID_ARG;
+    fa_status st = check_common(B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, dt);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) | reinterpret_cast<uintptr_t>(cu_seqlens_k) |
+         reinterpret_cast<uintptr_t>(seqused_k)) & 3u)
+        return FA_ERR_INVALID_ARG;
+    DeviceInfo di;
+    st = device_info(&di);
+    if (st != FA_OK) return st;
+    const bool bf16 = dt == FA_BF16;
+    // packed tensors: one batch entry of total rows
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap(&tq, q, 1, total_q, Hq, d, bf16) || !make_tmap(&tk, k, 1, total_k, Hkv, d, bf16) ||
+        !make_tmap(&tv, v, 1, total_k, Hkv, d, bf16))
+        return FA_ERR_CUDA;
+    fa::FwdParams p{};
+    p.o = o;
+    p.lse = lse;
+    p.cu_q = cu_seqlens_q;
+    p.cu_k = cu_seqlens_k;
+    p.used_k = seqused_k;
+    p.Sq_alloc = total_q;
+    p.B = B;
+    p.Sq = max_seqlen_q;
+    p.Sk = max_seqlen_k;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.group = Hq / Hkv;
+    const int unit = d == 128 ? 256 : 128;
+    p.num_m = (max_seqlen_q + unit - 1) / unit;
+    p.num_tiles = B * Hq * p.num_m;
+    p.chunk_heads = chunk_heads_for(B, Hq, p.group, max_seqlen_k, d);
     p.causal = causal ? 1 : 0;
     p.inject = take_inject();
     p.sl2 = scale * 1.4426950408889634f;

@@ -44,6 +44,15 @@ constexpr float kRescaleTau = 8.0f;
 struct FwdParams {
     void* o;
     float* lse;
+    // Packed variable-length batches (null for the dense [B, S, H, d] layout): the
+    // queries of sequence b are rows cu_q[b] .. cu_q[b+1]-1 of a [total_q, Hq, d]
+    // tensor, its keys rows cu_k[b] .. of [total_k, Hkv, d], of which the first
+    // used_k[b] (all when used_k is null) take part.  Sq / Sk are then the maximum
+    // lengths the grid is sized for.
+    const int* cu_q;
+    const int* cu_k;
+    const int* used_k;
+    int Sq_alloc;  // rows per batch entry of the q / o tensors (total_q when packed)
     int B, Sq, Sk, Hq, Hkv, group;
     int num_m;        // query blocks per head
     int num_tiles;    // B * Hq * num_m
@@ -129,16 +138,47 @@ __device__ __forceinline__ void fwd_decode(const FwdParams& p, int t, int& b, in
     m0 = mblk * UNIT_ROWS;
 }
 
-// Number of KV tiles a unit starting at query row m0 must visit.
+// One work unit: UNIT_ROWS query rows of one (batch entry, query head).
+struct FwdUnit {
+    int b, h, m0;          // m0: first query row of the unit within its sequence
+    int tb;                // batch coordinate in the TMA maps (0 for packed sequences)
+    int q_base, k_base;    // tensor row of the sequence's first query / key
+    int Sq, Sk;            // the sequence's query / key counts
+    int n;                 // KV tiles to visit
+    bool rows;             // the unit has query rows at all
+};
+
 template <int UNIT_ROWS>
-__device__ __forceinline__ int fwd_kv_tiles(const FwdParams& p, int m0)
+__device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int t)
 {
-    const int nk = (p.Sk + 127) / 128;
-    if (!p.causal) return nk;
-    const int last_row = min(m0 + UNIT_ROWS, p.Sq) - 1;
-    const long long maxcol = static_cast<long long>(last_row) + p.Sk - p.Sq;
-    if (maxcol < 0) return 0;
-    return min(nk, static_cast<int>(maxcol / 128) + 1);
+    FwdUnit u;
+    fwd_decode<UNIT_ROWS>(p, t, u.b, u.h, u.m0);
+    if (p.cu_q != nullptr) {
+        u.tb = 0;
+        u.q_base = p.cu_q[u.b];
+        u.k_base = p.cu_k[u.b];
+        const int sq = p.cu_q[u.b + 1] - u.q_base;
+        const int sk = p.used_k != nullptr ? p.used_k[u.b] : p.cu_k[u.b + 1] - u.k_base;
+        u.Sq = max(0, min(sq, p.Sq));
+        u.Sk = max(0, min(sk, p.Sk));
+    } else {
+        u.tb = u.b;
+        u.q_base = 0;
+        u.k_base = 0;
+        u.Sq = p.Sq;
+        u.Sk = p.Sk;
+    }
+    u.rows = u.m0 < u.Sq;
+    // KV tiles to visit: all of the sequence's keys, or with the causal mask (key j
+    // visible to query i iff j <= i + Sk - Sq) those up to the unit's last row's limit
+    const int nk = (u.Sk + 127) / 128;
+    u.n = u.rows ? nk : 0;
+    if (u.rows && p.causal) {
+        const int last_row = min(u.m0 + UNIT_ROWS, u.Sq) - 1;
+        const long long maxcol = static_cast<long long>(last_row) + u.Sk - u.Sq;
+        u.n = maxcol < 0 ? 0 : min(nk, static_cast<int>(maxcol / 128) + 1);
+    }
+    return u;
 }
 
 // ---------------------------------------------------------------------------------
@@ -159,15 +199,16 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
     uint32_t s_it = 0, tile_it = 0;
 
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-        int b, h, m0;
-        fwd_decode<C::UNIT_ROWS>(p, t, b, h, m0);
-        const int n = fwd_kv_tiles<C::UNIT_ROWS>(p, m0);
-        const int q0 = m0 + q * C::BM;  // first query row of this Q tile
+        const FwdUnit u = fwd_unit<C::UNIT_ROWS>(p, t);
+        if (!u.rows) continue;  // past the end of its (shorter) sequence: nothing to do
+        const int n = u.n, h = u.h;
+        const int q0 = u.m0 + q * C::BM;  // first query row of this Q tile
         const int row = q0 + r_in_tile;
-        const bool row_ok = row < p.Sq;
-        T* orow = reinterpret_cast<T*>(p.o) + ((static_cast<size_t>(b) * p.Sq + row) * p.Hq + h) * D;
-        float* lrow = p.lse + (static_cast<size_t>(b) * p.Hq + h) * p.Sq + row;
-        if (n == 0) {  // causal with Sq > Sk: no key is visible to any row of the unit
+        const bool row_ok = row < u.Sq;
+        const size_t orow_idx = static_cast<size_t>(u.tb) * p.Sq_alloc + u.q_base + row;
+        T* orow = reinterpret_cast<T*>(p.o) + (orow_idx * p.Hq + h) * D;
+        float* lrow = p.lse + (static_cast<size_t>(u.tb) * p.Hq + h) * p.Sq_alloc + u.q_base + row;
+        if (n == 0) {  // causal with Sq > Sk (or no keys): no key is visible to any row
             if (row_ok) {
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
@@ -178,8 +219,8 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
         }
         // columns >= lim are masked for this row; the tile-level test uses the first
         // row of the Q tile, which has the smallest limit
-        const int lim = p.causal ? min(p.Sk, row + p.Sk - p.Sq + 1) : p.Sk;
-        const int lim0 = p.causal ? min(p.Sk, q0 + p.Sk - p.Sq + 1) : p.Sk;
+        const int lim = p.causal ? min(u.Sk, row + u.Sk - u.Sq + 1) : u.Sk;
+        const int lim0 = p.causal ? min(u.Sk, q0 + u.Sk - u.Sq + 1) : u.Sk;
 
         float m_ref = -INFINITY;  // running reference max (log2 units)
         float l = 0.0f;           // running row sum against m_ref
@@ -394,9 +435,7 @@ struct FwdMma {
         uint32_t s_it[C::NQ] = {}, p_it[C::NQ] = {};
         uint32_t q_it = 0;
         for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-            int b, h, m0;
-            fwd_decode<C::UNIT_ROWS>(p, t, b, h, m0);
-            const int n = fwd_kv_tiles<C::UNIT_ROWS>(p, m0);
+            const int n = fwd_unit<C::UNIT_ROWS>(p, t).n;
             if (n == 0) continue;
             if (!wait(bar(C::B_Q_FULL), q_it & 1u, W_FWD_Q_FULL)) return;
             ++q_it;
@@ -524,10 +563,10 @@ struct FwdLoad {
         filled[slot] = static_cast<int>(round);
         return true;
     }
-    __device__ bool load_kv(const CUtensorMap* tm, int j, int hkv, int b)
+    __device__ bool load_kv(const CUtensorMap* tm, int row0, int hkv, int b)
     {
         for (int c = 0; c < C::KCH; ++c)
-            if (!load_chunk(tm, j * C::BN, c * 128, hkv, b)) return false;
+            if (!load_chunk(tm, row0, c * 128, hkv, b)) return false;
         return true;
     }
 
@@ -537,30 +576,32 @@ struct FwdLoad {
         inject = p.inject;
         uint32_t q_it = 0;
         for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-            int b, h, m0;
-            fwd_decode<C::UNIT_ROWS>(p, t, b, h, m0);
-            const int n = fwd_kv_tiles<C::UNIT_ROWS>(p, m0);
+            const FwdUnit u = fwd_unit<C::UNIT_ROWS>(p, t);
+            const int n = u.n, b = u.tb;
             if (n == 0) continue;
-            const int hkv = h / p.group;
+            const int hkv = u.h / p.group;
+            // rows past the sequence's end (the next sequence's, or out of range) are
+            // loaded too: their scores are masked, their outputs never stored
+            auto krow = [&](int j) { return u.k_base + j * C::BN; };
             if (!wait_bar(bar(C::B_Q_EMPTY), (q_it & 1u) ^ 1u, ctl, W_FWD_Q_EMPTY)) return;
             mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_BYTES);
             for (int q = 0; q < C::NQ; ++q)
                 for (int blk = 0; blk < D / 64; ++blk)
-                    tma_load_4d(sQ + q * C::QTILE + blk * 16384u, tmQ, bar(C::B_Q_FULL), blk * 64, h,
-                                m0 + q * C::BM, b);
+                    tma_load_4d(sQ + q * C::QTILE + blk * 16384u, tmQ, bar(C::B_Q_FULL), blk * 64, u.h,
+                                u.q_base + u.m0 + q * C::BM, b);
             q_round = static_cast<int>(q_it);
             ++q_it;
             if constexpr (C::NQ == 2) {
                 for (int j = 0; j < n; ++j) {
-                    if (!load_kv(tmK, j, hkv, b)) return;
-                    if (!load_kv(tmV, j, hkv, b)) return;
+                    if (!load_kv(tmK, krow(j), hkv, b)) return;
+                    if (!load_kv(tmV, krow(j), hkv, b)) return;
                 }
             } else {
                 for (int j = 0; j < 2 && j < n; ++j)
-                    if (!load_kv(tmK, j, hkv, b)) return;
+                    if (!load_kv(tmK, krow(j), hkv, b)) return;
                 for (int j = 0; j < n; ++j) {
-                    if (!load_kv(tmV, j, hkv, b)) return;
-                    if (j + 2 < n && !load_kv(tmK, j + 2, hkv, b)) return;
+                    if (!load_kv(tmV, krow(j), hkv, b)) return;
+                    if (j + 2 < n && !load_kv(tmK, krow(j + 2), hkv, b)) return;
                 }
             }
         }

@@ -67,6 +67,26 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  fa_dtype dt, fa_stream stream);
 
 /*
+ * Forward over a packed batch of variable-length sequences (the varlen row of
+ * "[RFC] FA4 -- head_dim=256 & head_dim=512", Phase 1: cu_seqlens and seqused_k).
+ * Sequence b's queries are rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 of
+ * q [total_q, Hq, d] (o has the same layout), its keys rows cu_seqlens_k[b] ..
+ * cu_seqlens_k[b+1]-1 of k, v [total_k, Hkv, d], of which the first seqused_k[b]
+ * take part (seqused_k may be NULL: all of them).  lse is float32 [Hq, total_q].
+ * cu_seqlens_q / cu_seqlens_k are device int32 arrays of B+1 nondecreasing offsets
+ * starting at 0 and ending at total_q / total_k; seqused_k a device int32 array of
+ * B counts.  max_seqlen_q / max_seqlen_k bound the sequence lengths (the grid is
+ * sized by them; longer sequences are cut to them).  Each sequence is an
+ * independent attention problem with the causal mask aligned to its own bottom
+ * right.  Same dtypes, alignment, ownership and error behaviour as fa_fwd; the
+ * offsets live on the device and are not checked by the host.
+ */
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, const int* seqused_k, int B,
+                        int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv,
+                        int d, int causal, float scale, fa_dtype dt, fa_stream stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for these sizes: the row terms
  * D = rowsum(dO * O), the log2-domain LSE copy and the float32 dQ accumulator.
  */
