@@ -8,6 +8,8 @@ library's CUDA kernels.  The functions carry the C names:
     fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
                   seqused_k=None, causal=False, scale=None) -> (o, lse)
     fa_bwd(q, k, v, o, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
+    fa_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                  max_seqlen_k, seqused_k=None, causal=False, scale=None) -> (dq, dk, dv)
     fa_bwd_workspace_size(B, Sq, Hq, d) -> int
     fa_bwd_noalloc(q, k, v, o, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
     fa_status_string(code) -> str
@@ -29,7 +31,7 @@ import torch
 from . import _lib
 
 __all__ = [
-    "FAError", "fa_fwd", "fa_fwd_varlen", "fa_bwd", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
+    "FAError", "fa_fwd", "fa_fwd_varlen", "fa_bwd", "fa_bwd_varlen", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
     "fa_last_device_status", "fa_clear_device_status", "fa_debug_inject", "fa_debug_exp2",
 ]
 
@@ -160,6 +162,39 @@ def fa_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = No
                               float(scale), _dtype_code(q), workspace.data_ptr(),
                               workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _raise(code, "fa_bwd")
+    return dq, dk, dv
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                  max_seqlen_k: int, seqused_k=None, causal: bool = False, scale: float | None = None,
+                  dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Backward over packed variable-length sequences (layouts as fa_fwd_varlen)
+    -> (dq [total_q,Hq,d], dk, dv [total_k,Hkv,d])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _check(t, n, q.dtype)
+    _check(lse, "lse", torch.float32)
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)) + (
+            (("seqused_k", seqused_k),) if seqused_k is not None else ()):
+        if t.device.type != "cuda" or t.dtype != torch.int32 or not t.is_contiguous():
+            raise ValueError(f"fa: {name} must be a contiguous CUDA int32 tensor")
+    B = cu_seqlens_q.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = fa_bwd_workspace_size(B, int(max_seqlen_q), Hq, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    code = _lib.load().fa_bwd_varlen(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
+        seqused_k.data_ptr() if seqused_k is not None else None, B, int(max_seqlen_q), int(max_seqlen_k),
+        total_q, total_k, Hq, Hkv, d, int(bool(causal)), float(scale), _dtype_code(q), workspace.data_ptr(),
+        workspace.numel(), _stream_ptr(stream))
+    _raise(code, "fa_bwd_varlen")
     return dq, dk, dv
 
 

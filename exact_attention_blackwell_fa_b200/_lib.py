@@ -25,6 +25,8 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (_sz, [_ci, _ci, _ci, _ci]),
     "fa_bwd": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci,
                      _ci, _cf, _ci, _vp, _sz, _vp]),
+    "fa_bwd_varlen": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci,
+                            _ci, _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp, _sz, _vp]),
     "fa_bwd_noalloc": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
                              _ci, _ci, _ci, _cf, _ci, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_ci]),

@@ -301,10 +301,14 @@ size_t fa_bwd_workspace_size(int B, int Sq, int Hq, int d)
     return fa::bwd_workspace_bytes(B, Sq, Hq, d);
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                 const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq,
-                 int Hkv, int d, int causal, float scale, fa_dtype dt, void* workspace,
-                 size_t workspace_bytes, fa_stream stream)
+// The backward for B batch entries of (at most) Sq queries and Sk keys; the q-side
+// tensors hold Sq_alloc rows per entry and the k-side Sk_alloc (packed sequences:
+// one entry of total rows, with cu_q / cu_k / used_k describing the sequences).
+static fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dout, void* dq, void* dk, void* dv, const int* cu_q, const int* cu_k,
+                            const int* used_k, int B, int Sq, int Sk, int Sq_alloc, int Sk_alloc, int TB,
+                            int Hq, int Hkv, int d, int causal, float scale, fa_dtype dt, void* workspace,
+                            size_t workspace_bytes, fa_stream stream)
 {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
         return FA_ERR_INVALID_ARG;
@@ -321,8 +325,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     const bool bf16 = dt == FA_BF16;
     const int kv_rows = d == 128 ? 128 : 64;  // keys per backward work unit
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_tmap(&tq, q, B, Sq, Hq, d, bf16) || !make_tmap(&tk, k, B, Sk, Hkv, d, bf16, kv_rows) ||
-        !make_tmap(&tv, v, B, Sk, Hkv, d, bf16, kv_rows) || !make_tmap(&tdo, dout, B, Sq, Hq, d, bf16))
+    if (!make_tmap(&tq, q, TB, Sq_alloc, Hq, d, bf16) || !make_tmap(&tk, k, TB, Sk_alloc, Hkv, d, bf16, kv_rows) ||
+        !make_tmap(&tv, v, TB, Sk_alloc, Hkv, d, bf16, kv_rows) || !make_tmap(&tdo, dout, TB, Sq_alloc, Hq, d, bf16))
         return FA_ERR_CUDA;
     fa::BwdParams p{};
     p.o = o;
@@ -337,6 +341,11 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     p.dq = dq;
     p.dk = dk;
     p.dv = dv;
+    p.cu_q = cu_q;
+    p.cu_k = cu_k;
+    p.used_k = used_k;
+    p.Sq_alloc = Sq_alloc;
+    p.Sk_alloc = Sk_alloc;
     p.B = B;
     p.Sq = Sq;
     p.Sk = Sk;
@@ -364,6 +373,30 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                     : launch_bwd_d256<false>(tq, tk, tv, tdo, p, di.sm_count, s);
     return bf16 ? launch_bwd_d128<true>(tq, tk, tv, tdo, p, di.sm_count, s)
                 : launch_bwd_d128<false>(tq, tk, tv, tdo, p, di.sm_count, s);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq,
+                 int Hkv, int d, int causal, float scale, fa_dtype dt, void* workspace,
+                 size_t workspace_bytes, fa_stream stream)
+{
+    return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, nullptr, nullptr, nullptr, B, Sq, Sk, Sq, Sk, B, Hq, Hkv, d,
+                      causal, scale, dt, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                        const int* cu_seqlens_k, const int* seqused_k, int B, int max_seqlen_q,
+                        int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, int causal,
+                        float scale, fa_dtype dt, void* workspace, size_t workspace_bytes, fa_stream stream)
+{
+    if (!cu_seqlens_q || !cu_seqlens_k || total_q < 1 || total_k < 1) return FA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) | reinterpret_cast<uintptr_t>(cu_seqlens_k) |
+         reinterpret_cast<uintptr_t>(seqused_k)) & 3u)
+        return FA_ERR_INVALID_ARG;
+    return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, seqused_k, B, max_seqlen_q,
+                      max_seqlen_k, total_q, total_k, 1, Hq, Hkv, d, causal, scale, dt, workspace, workspace_bytes,
+                      stream);
 }
 
 const char* fa_status_string(fa_status s)

@@ -52,6 +52,14 @@ struct BwdParams {
     void* dq;
     void* dk;
     void* dv;
+    // Packed variable-length batches (null for the dense layout): sequence b's
+    // queries are rows cu_q[b] .. of the [total_q, Hq, d] tensors, its keys rows
+    // cu_k[b] .. of [total_k, Hkv, d], the first used_k[b] of them taking part.
+    // Sq / Sk are then the maximum lengths; the workspace stays dense per sequence.
+    const int* cu_q;
+    const int* cu_k;
+    const int* used_k;
+    int Sq_alloc, Sk_alloc;  // rows per batch entry of the q- / k-side tensors
     int B, Sq, Sk, Hq, Hkv, group, Sq_pad;
     int num_n;        // key blocks per KV head
     int num_m;        // query blocks per query head
@@ -67,6 +75,33 @@ enum : uint32_t {
     W_BWD_DQ_FULL, W_BWD_DQ_EMPTY, W_BWD_DKV_FINAL, W_BWD_DRAIN, W_BWD_SMEM_ALIGN
 };
 
+// Rows of batch entry b: the TMA batch coordinate, the tensor rows of its first
+// query and key, and its query / key counts.
+struct BwdSeq {
+    int tb, q_base, k_base, Sq, Sk;
+};
+
+__device__ __forceinline__ BwdSeq bwd_seq(const BwdParams& p, int b)
+{
+    BwdSeq s;
+    if (p.cu_q != nullptr) {
+        s.tb = 0;
+        s.q_base = p.cu_q[b];
+        s.k_base = p.cu_k[b];
+        const int sq = p.cu_q[b + 1] - s.q_base;
+        const int sk = p.used_k != nullptr ? p.used_k[b] : p.cu_k[b + 1] - s.k_base;
+        s.Sq = max(0, min(sq, p.Sq));
+        s.Sk = max(0, min(sk, p.Sk));
+    } else {
+        s.tb = b;
+        s.q_base = 0;
+        s.k_base = 0;
+        s.Sq = p.Sq;
+        s.Sk = p.Sk;
+    }
+    return s;
+}
+
 // ---------------------------------------------------------------------------------
 // 1. preprocess: one warp per padded query row (b, h, i)
 // ---------------------------------------------------------------------------------
@@ -80,9 +115,11 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p)
     const int bh = static_cast<int>(row / p.Sq_pad);
     const int i = static_cast<int>(row - static_cast<long long>(bh) * p.Sq_pad);
     const int b = bh / p.Hq, h = bh - b * p.Hq;
+    const BwdSeq sq = bwd_seq(p, b);
+    const size_t trow = static_cast<size_t>(sq.tb) * p.Sq_alloc + sq.q_base + i;  // tensor row
     float acc = 0.0f;
-    if (i < p.Sq) {
-        const size_t off = ((static_cast<size_t>(b) * p.Sq + i) * p.Hq + h) * D + lane * (D / 32);
+    if (i < sq.Sq) {
+        const size_t off = (trow * p.Hq + h) * D + lane * (D / 32);
         constexpr int NW = D / 64;  // 32-bit words per lane (two 16-bit values each)
         uint32_t ow[NW], dw[NW];
         if constexpr (NW == 2) {
@@ -108,8 +145,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p)
     if (lane == 0) {
         p.Dv[row] = acc;
         float l2 = INFINITY;
-        if (i < p.Sq) {
-            const float lse = p.lse[static_cast<size_t>(bh) * p.Sq + i];
+        if (i < sq.Sq) {
+            const float lse = p.lse[(static_cast<size_t>(sq.tb) * p.Hq + h) * p.Sq_alloc + sq.q_base + i];
             if (lse != -INFINITY) l2 = lse * 1.4426950408889634f;
         }
         p.L2[row] = l2;
@@ -133,8 +170,11 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p)
     const long long bi = row / p.Hq;
     const int i = static_cast<int>(bi % p.Sq);
     const int b = static_cast<int>(bi / p.Sq);
+    const BwdSeq sq = bwd_seq(p, b);
+    if (i >= sq.Sq) return;
+    const size_t trow = static_cast<size_t>(sq.tb) * p.Sq_alloc + sq.q_base + i;
     const float* src = p.dqacc + ((static_cast<size_t>(b) * p.Hq + h) * p.Sq_pad + i) * D + lane * (D / 32);
-    uint16_t* dst = static_cast<uint16_t*>(p.dq) + static_cast<size_t>(row) * D + lane * (D / 32);
+    uint16_t* dst = static_cast<uint16_t*>(p.dq) + (trow * p.Hq + h) * D + lane * (D / 32);
     if constexpr (D == 128) {
         const float4 a = *reinterpret_cast<const float4*>(src);
         *reinterpret_cast<uint2*>(dst) =
@@ -158,9 +198,9 @@ struct BwdCfg {
     // 13: TMA, 14-15: idle (they complete the fourth warpgroup for setmaxnreg)
     static constexpr int THREADS = 512;
     static constexpr int DQ_WARP = 8, MMA_WARP = 12, LOAD_WARP = 13;
-    // registers per thread: launched at 128; the MMA/TMA warpgroup gives 24 of them to
+    // registers per thread: launched at 128; the MMA/TMA warpgroup gives 16 of them to
     // the dQ warpgroup, which then holds a whole 128-column dQ^T row in registers
-    static constexpr uint32_t REG_LAUNCH = 128, REG_DQ = 152, REG_CTRL = 104;
+    static constexpr uint32_t REG_LAUNCH = 128, REG_DQ = 144, REG_CTRL = 112;
     static_assert(8 * 32 * REG_LAUNCH + 4 * 32 * REG_DQ + 4 * 32 * REG_CTRL <= THREADS * REG_LAUNCH,
                   "register split exceeds the launch budget");
     // lane 0 of the MMA warp issues alone (the converged, elected-lane form measured
@@ -190,6 +230,8 @@ struct BwdCfg {
 
 struct BwdUnit {
     int b, hkv, n, m_start, nm, T;
+    int tb, q_base, k_base, Sq, Sk;  // the batch entry's rows (see BwdSeq)
+    bool keys;                       // the unit's key block holds keys of its sequence
 };
 
 __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int t)
@@ -206,14 +248,22 @@ __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int t)
     u.b = bh / p.Hkv;
     u.hkv = bh - u.b * p.Hkv;
     u.n = nb;
+    const BwdSeq sq = bwd_seq(p, u.b);
+    u.tb = sq.tb;
+    u.q_base = sq.q_base;
+    u.k_base = sq.k_base;
+    u.Sq = sq.Sq;
+    u.Sk = sq.Sk;
+    u.keys = u.n * 128 < u.Sk;
+    const int num_m = (u.Sq + 127) / 128;
     int ms = 0;
     if (p.causal) {
-        const long long imin = static_cast<long long>(u.n) * 128 - (p.Sk - p.Sq);
+        const long long imin = static_cast<long long>(u.n) * 128 - (u.Sk - u.Sq);
         ms = imin <= 0 ? 0 : static_cast<int>(imin / 128);
-        if (ms > p.num_m) ms = p.num_m;
+        if (ms > num_m) ms = num_m;
     }
     u.m_start = ms;
-    u.nm = p.num_m - ms;
+    u.nm = u.keys ? num_m - ms : 0;
     u.T = p.group * u.nm;
     return u;
 }
@@ -245,14 +295,35 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
     uint32_t it = 0, unit_it = 0;
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
         const BwdUnit u = bwd_decode(p, ui);
+        if (!u.keys) continue;  // past the end of its sequence's keys
         const int j = u.n * 128 + t;  // key row
+        // offset of key row j's dK / dV row
+        auto grad_off = [&]() {
+            return ((static_cast<size_t>(u.tb) * p.Sk_alloc + u.k_base + j) * p.Hkv + u.hkv) * C::D;
+        };
+        if (u.T == 0) {  // keys that no query of the sequence sees: zero gradients
+            if (j < u.Sk) {
+                T* const dvrow = static_cast<T*>(p.dv) + grad_off();
+                T* const dkrow = static_cast<T*>(p.dk) + grad_off();
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                for (int c = 2 * half; c < 2 * half + 2; ++c)
+                    for (int x = 0; x < 4; ++x) {
+                        reinterpret_cast<uint4*>(dvrow + c * 32)[x] = z;
+                        reinterpret_cast<uint4*>(dkrow + c * 32)[x] = z;
+                    }
+            }
+            continue;
+        }
         for (int s = 0; s < u.T; ++s, ++it) {
             int h, m;
             bwd_step(p, u, s, h, m);
             const uint32_t rows = sRows + (it & 1) * C::ROWS_BYTES;  // L2[128] then D[128]
-            // key j is visible to query i iff j <= i + (Sk - Sq)
-            const bool masked = p.causal && (u.n * 128 + 127 > m * 128 + p.Sk - p.Sq);
-            const int jlim = j - (p.Sk - p.Sq) - m * 128 - q0;  // visible iff column c >= jlim
+            // key j is visible to query i iff j <= i + (Sk - Sq) (causal) and j < Sk: the
+            // key block's rows past the sequence's keys (zeros, or the next sequence's
+            // rows of a packed batch) get P = 0
+            const bool masked = (p.causal && (u.n * 128 + 127 > m * 128 + u.Sk - u.Sq)) || (u.n * 128 + 128 > u.Sk);
+            int jlim = p.causal ? j - (u.Sk - u.Sq) - m * 128 - q0 : -(1 << 30);  // visible iff column c >= jlim
+            if (j >= u.Sk) jlim = 1 << 30;
             // the Q-tile barrier also covers the staged row terms
             if (!warp_wait<true, true>(bar(C::B_Q_FULL + (it & 1)), (it >> 1) & 1u, ctl, W_BWD_Q_FULL)) return;
             if (!warp_wait<true, true>(bar(C::B_S_FULL), it & 1u, ctl, W_BWD_S_FULL)) return;
@@ -345,10 +416,9 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
         if (!warp_wait<true, true>(bar(C::B_DKV_FINAL), unit_it & 1u, ctl, W_BWD_DKV_FINAL)) return;
         ++unit_it;
         tc_fence_after();
-        const bool row_ok = j < p.Sk;
-        const size_t off = ((static_cast<size_t>(u.b) * p.Sk + j) * p.Hkv + u.hkv) * C::D;
-        T* dvrow = static_cast<T*>(p.dv) + off;
-        T* dkrow = static_cast<T*>(p.dk) + off;
+        const bool row_ok = j < u.Sk;
+        T* const dvrow = static_cast<T*>(p.dv) + grad_off();
+        T* const dkrow = static_cast<T*>(p.dk) + grad_off();
 #pragma unroll 1
         for (int which = 0; which < 2; ++which) {
             const float mul = which == 0 ? 1.0f : p.scale;
@@ -547,8 +617,8 @@ struct BwdLoad {
             if (u.T == 0) continue;
             if (!wait_bar_inl(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_BWD_KV_EMPTY)) return;
             mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::TILE);
-            tile(base + C::OFF_K, tmK, bar(C::B_KV_FULL), u.hkv, u.n * 128, u.b);
-            tile(base + C::OFF_V, tmV, bar(C::B_KV_FULL), u.hkv, u.n * 128, u.b);
+            tile(base + C::OFF_K, tmK, bar(C::B_KV_FULL), u.hkv, u.k_base + u.n * 128, u.tb);
+            tile(base + C::OFF_V, tmV, bar(C::B_KV_FULL), u.hkv, u.k_base + u.n * 128, u.tb);
             kv_round = static_cast<int>(unit_it);
             ++unit_it;
             for (int s = 0; s < u.T; ++s, ++it) {
@@ -558,7 +628,7 @@ struct BwdLoad {
                 const uint32_t ph = ((it >> 1) & 1u) ^ 1u;
                 if (!wait_bar_inl(bar(C::B_Q_EMPTY + st), ph, ctl, W_BWD_Q_EMPTY)) return;
                 mbar_arrive_expect_tx(bar(C::B_Q_FULL + st), C::TILE + C::ROWS_BYTES);
-                tile(base + C::OFF_Q + st * C::TILE, tmQ, bar(C::B_Q_FULL + st), h, m * 128, u.b);
+                tile(base + C::OFF_Q + st * C::TILE, tmQ, bar(C::B_Q_FULL + st), h, u.q_base + m * 128, u.tb);
                 {
                     const size_t rb = (static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad +
                                       static_cast<size_t>(m) * 128;
@@ -569,7 +639,7 @@ struct BwdLoad {
                 q_round[st] = static_cast<int>(it >> 1);
                 if (!wait_bar_inl(bar(C::B_DO_EMPTY + st), ph, ctl, W_BWD_DO_EMPTY)) return;
                 mbar_arrive_expect_tx(bar(C::B_DO_FULL + st), C::TILE);
-                tile(base + C::OFF_DO + st * C::TILE, tmDO, bar(C::B_DO_FULL + st), h, m * 128, u.b);
+                tile(base + C::OFF_DO + st * C::TILE, tmDO, bar(C::B_DO_FULL + st), h, u.q_base + m * 128, u.tb);
                 do_round[st] = static_cast<int>(it >> 1);
             }
         }

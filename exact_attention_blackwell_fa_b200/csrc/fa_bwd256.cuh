@@ -86,14 +86,22 @@ __device__ __forceinline__ BwdUnit bwd256_decode(const BwdParams& p, int t)
     u.b = bh / p.Hkv;
     u.hkv = bh - u.b * p.Hkv;
     u.n = nb;
+    const BwdSeq sq = bwd_seq(p, u.b);
+    u.tb = sq.tb;
+    u.q_base = sq.q_base;
+    u.k_base = sq.k_base;
+    u.Sq = sq.Sq;
+    u.Sk = sq.Sk;
+    u.keys = u.n * 64 < u.Sk;
+    const int num_m = (u.Sq + 127) / 128;
     int ms = 0;
     if (p.causal) {
-        const long long imin = static_cast<long long>(u.n) * 64 - (p.Sk - p.Sq);
+        const long long imin = static_cast<long long>(u.n) * 64 - (u.Sk - u.Sq);
         ms = imin <= 0 ? 0 : static_cast<int>(imin / 128);
-        if (ms > p.num_m) ms = p.num_m;
+        if (ms > num_m) ms = num_m;
     }
     u.m_start = ms;
-    u.nm = p.num_m - ms;
+    u.nm = u.keys ? num_m - ms : 0;
     u.T = p.group * u.nm;
     return u;
 }
@@ -128,13 +136,27 @@ __device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base,
     uint32_t it = 0, unit_it = 0;
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
         const BwdUnit u = bwd256_decode(p, ui);
+        if (!u.keys) continue;  // past the end of its sequence's keys
+        // dV^T / dK^T element of head-dim column (hf * 128 + t) for key `key` of the unit
+        auto grad_off = [&](int key, int hf) {
+            return ((static_cast<size_t>(u.tb) * p.Sk_alloc + u.k_base + key) * p.Hkv + u.hkv) * C::D + hf * 128 + t;
+        };
+        if (u.T == 0) {  // keys that no query of the sequence sees: zero gradients
+            T* dst = static_cast<T*>(half == 0 ? p.dv : p.dk);
+            for (int key = u.n * 64; key < min(u.n * 64 + 64, u.Sk); ++key)
+                for (int hf = 0; hf < 2; ++hf) dst[grad_off(key, hf)] = static_cast<T>(0.0f);
+            continue;
+        }
         for (int s = 0; s < u.T; ++s, ++it) {
             int h, m;
             bwd_step(p, u, s, h, m);
             const int i = m * 128 + t;  // query row
-            // key n*64 + c is visible iff c <= lim
-            const int lim = i + (p.Sk - p.Sq) - u.n * 64;
-            const bool masked = p.causal && (u.n * 64 + 63 > m * 128 + p.Sk - p.Sq);
+            // key n*64 + c is visible iff c <= lim: (causal) c <= i + Sk - Sq - n*64, and
+            // c < Sk - n*64 (rows past the sequence's keys: zeros, or the next sequence's
+            // rows of a packed batch)
+            const int klim = u.Sk - 1 - u.n * 64;
+            const int lim = p.causal ? min(i + (u.Sk - u.Sq) - u.n * 64, klim) : klim;
+            const bool masked = (p.causal && (u.n * 64 + 63 > m * 128 + u.Sk - u.Sq)) || (u.n * 64 + 64 > u.Sk);
             if (!warp_wait<true>(bar(C::B_Q_FULL), it & 1u, ctl, W_B256_Q_FULL)) return;
             float l2, dval;
             asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l2) : "r"(base + C::OFF_ROWS + t * 4u));
@@ -206,11 +228,7 @@ __device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base,
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const int key = u.n * 64 + cc * 32 + c;
-                        if (key < p.Sk) {
-                            const size_t off =
-                                ((static_cast<size_t>(u.b) * p.Sk + key) * p.Hkv + u.hkv) * C::D + hf * 128 + t;
-                            dst[off] = static_cast<T>(__uint_as_float(r[c]) * mul);
-                        }
+                        if (key < u.Sk) dst[grad_off(key, hf)] = static_cast<T>(__uint_as_float(r[c]) * mul);
                     }
                 }
             }
@@ -368,8 +386,10 @@ struct Bwd256Load {
             if (!wait_bar_inl(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_B256_KV_EMPTY)) return;
             mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::KV_BYTES);
             for (int blk = 0; blk < 4; ++blk) {
-                tma_load_4d(base + C::OFF_K + blk * C::KV_BLK, tmK, bar(C::B_KV_FULL), blk * 64, u.hkv, u.n * 64, u.b);
-                tma_load_4d(base + C::OFF_V + blk * C::KV_BLK, tmV, bar(C::B_KV_FULL), blk * 64, u.hkv, u.n * 64, u.b);
+                tma_load_4d(base + C::OFF_K + blk * C::KV_BLK, tmK, bar(C::B_KV_FULL), blk * 64, u.hkv,
+                            u.k_base + u.n * 64, u.tb);
+                tma_load_4d(base + C::OFF_V + blk * C::KV_BLK, tmV, bar(C::B_KV_FULL), blk * 64, u.hkv,
+                            u.k_base + u.n * 64, u.tb);
             }
             kv_round = static_cast<int>(unit_it);
             ++unit_it;
@@ -380,7 +400,8 @@ struct Bwd256Load {
                 if (!wait_bar_inl(bar(C::B_Q_EMPTY), ph, ctl, W_B256_Q_EMPTY)) return;
                 mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_BYTES + C::ROWS_BYTES);
                 for (int blk = 0; blk < 4; ++blk)
-                    tma_load_4d(base + C::OFF_Q + blk * C::Q_BLK, tmQ, bar(C::B_Q_FULL), blk * 64, h, m * 128, u.b);
+                    tma_load_4d(base + C::OFF_Q + blk * C::Q_BLK, tmQ, bar(C::B_Q_FULL), blk * 64, h,
+                                u.q_base + m * 128, u.tb);
                 {
                     const size_t rb = (static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + static_cast<size_t>(m) * 128;
                     bulk_load(base + C::OFF_ROWS, p.L2 + rb, 512, bar(C::B_Q_FULL));
@@ -390,7 +411,8 @@ struct Bwd256Load {
                 if (!wait_bar_inl(bar(C::B_DO_EMPTY), ph, ctl, W_B256_DO_EMPTY)) return;
                 mbar_arrive_expect_tx(bar(C::B_DO_FULL), C::Q_BYTES);
                 for (int blk = 0; blk < 4; ++blk)
-                    tma_load_4d(base + C::OFF_DO + blk * C::Q_BLK, tmDO, bar(C::B_DO_FULL), blk * 64, h, m * 128, u.b);
+                    tma_load_4d(base + C::OFF_DO + blk * C::Q_BLK, tmDO, bar(C::B_DO_FULL), blk * 64, h,
+                                u.q_base + m * 128, u.tb);
                 do_round = static_cast<int>(it);
             }
         }

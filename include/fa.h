@@ -105,6 +105,21 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  fa_dtype dt, void* workspace, size_t workspace_bytes, fa_stream stream);
 
 /*
+ * Backward over a packed batch of variable-length sequences: the inputs as for
+ * fa_fwd_varlen (o, dout and dq [total_q, Hq, d]; dk, dv [total_k, Hkv, d]; lse
+ * [Hq, total_q] from fa_fwd_varlen) and the workspace of
+ * fa_bwd_workspace_size(B, max_seqlen_q, Hq, d).  Gradient rows of keys past
+ * seqused_k[b] (allocated but not taking part) are not written; rows of keys that
+ * take part but that no query sees are written as zeros.  Same ownership, ordering
+ * and error behaviour as fa_bwd.
+ */
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                        const int* cu_seqlens_k, const int* seqused_k, int B, int max_seqlen_q,
+                        int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, int causal,
+                        float scale, fa_dtype dt, void* workspace, size_t workspace_bytes, fa_stream stream);
+
+/*
  * Backward that allocates nothing and takes no workspace: the same computation as
  * fa_bwd, with its scratch (the row terms and the float32 dQ accumulator) kept in a
  * fixed device array built into the library.  The paper has no counterpart to this
