@@ -183,6 +183,9 @@ def main():
     ap.add_argument("--hd", type=int, default=None)
     ap.add_argument("--causal", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--varlen", default=None,
+                    help="comma-separated sequence lengths: one packed batch of these sequences "
+                         "(fa_fwd_varlen / fa_bwd_varlen) instead of the dense workload")
     args = ap.parse_args()
     if args.batch is not None:
         WORKLOAD["B"] = args.batch
@@ -200,16 +203,26 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     W = WORKLOAD
-    f_fwd, f_bwd = flops(W["B"], W["S"], W["S"], W["H"], W["d"], W["causal"])
-    config = {"workload": f"attention fwd+bwd bf16 B={W['B']} S={W['S']} H={W['H']} "
-                          f"Hkv={W['Hkv']} d={W['d']} "
-                          f"{'causal' if W['causal'] else 'non-causal'}",
+    lens = [int(x) for x in args.varlen.split(",")] if args.varlen else None
+    if lens:
+        W["B"], W["S"] = len(lens), max(lens)
+        f_fwd = sum(flops(1, L, L, W["H"], W["d"], W["causal"])[0] for L in lens)
+        f_bwd = 2.5 * f_fwd
+        wl = (f"attention fwd+bwd bf16 varlen packed lens={','.join(map(str, lens))} H={W['H']} "
+              f"Hkv={W['Hkv']} d={W['d']} {'causal' if W['causal'] else 'non-causal'}")
+    else:
+        f_fwd, f_bwd = flops(W["B"], W["S"], W["S"], W["H"], W["d"], W["causal"])
+        wl = (f"attention fwd+bwd bf16 B={W['B']} S={W['S']} H={W['H']} Hkv={W['Hkv']} d={W['d']} "
+              f"{'causal' if W['causal'] else 'non-causal'}")
+    config = {"workload": wl,
               "B": W["B"], "seq_len": W["S"], "heads": W["H"], "kv_heads": W["Hkv"],
               "head_dim": W["d"],
               "causal": W["causal"], "global_batch": W["B"] * world,
               "parallelism": f"replicas x{world} (independent batches, no collective)",
               "l2": ("inputs larger than L2 (each of Q, O, dO is "
-                     f"{W['B'] * W['S'] * W['H'] * W['d'] * 2 / 2**20:.0f} MiB)")}
+                     f"{(sum(lens) if lens else W['B'] * W['S']) * W['H'] * W['d'] * 2 / 2**20:.0f} MiB)")}
+    if lens:
+        config["seq_lens"] = lens
 
     if args.impl == "reference":
         if rank != 0:
@@ -244,21 +257,45 @@ def main():
     dev = torch.device("cuda", local_rank if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
 
-    shape = Shape(W["B"], W["S"], W["S"], W["H"], W["Hkv"], W["d"])
-    q, k, v, do = make_inputs(shape, seed=rank, device=dev, with_dout=True)
     do_bwd = not args.fwd_only
+    if lens:
+        total = sum(lens)
+        q, k, v, do = (t[0] for t in make_inputs(Shape(1, total, total, W["H"], W["Hkv"], W["d"]), seed=rank,
+                                                 device=dev, with_dout=True))
+        cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0)), dtype=torch.int32, device=dev)
+        lse = torch.empty(W["H"], total, dtype=torch.float32, device=dev)
+    else:
+        shape = Shape(W["B"], W["S"], W["S"], W["H"], W["Hkv"], W["d"])
+        q, k, v, do = make_inputs(shape, seed=rank, device=dev, with_dout=True)
+        lse = torch.empty(W["B"], W["H"], W["S"], dtype=torch.float32, device=dev)
     o = torch.empty_like(q)
-    lse = torch.empty(W["B"], W["H"], W["S"], dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(fa.fa_bwd_workspace_size(W["B"], W["S"], W["H"], W["d"]), dtype=torch.uint8,
                      device=dev)
     stream = torch.cuda.current_stream(dev)
+    main_bufs = dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws)
+
+    # the forward and backward calls through the public API, on a set of buffers
+    def run_fwd(t, st):
+        if lens:
+            fa.fa_fwd_varlen(t["q"], t["k"], t["v"], cu, cu, W["S"], W["S"], causal=W["causal"], out=t["o"],
+                             lse=t["lse"], stream=st)
+        else:
+            fa.fa_fwd(t["q"], t["k"], t["v"], causal=W["causal"], out=t["o"], lse=t["lse"], stream=st)
+
+    def run_bwd(t, st):
+        if lens:
+            fa.fa_bwd_varlen(t["q"], t["k"], t["v"], t["o"], t["lse"], t["do"], cu, cu, W["S"], W["S"],
+                             causal=W["causal"], dq=t["dq"], dk=t["dk"], dv=t["dv"], workspace=t["ws"],
+                             stream=st)
+        else:
+            fa.fa_bwd(t["q"], t["k"], t["v"], t["o"], t["lse"], t["do"], causal=W["causal"], dq=t["dq"],
+                      dk=t["dk"], dv=t["dv"], workspace=t["ws"], stream=st)
 
     def step():
-        fa.fa_fwd(q, k, v, causal=W["causal"], out=o, lse=lse, stream=stream)
+        run_fwd(main_bufs, stream)
         if do_bwd:
-            fa.fa_bwd(q, k, v, o, lse, do, causal=W["causal"], dq=dq, dk=dk, dv=dv,
-                      workspace=ws, stream=stream)
+            run_bwd(main_bufs, stream)
 
     def barrier():
         if world > 1:
@@ -284,11 +321,10 @@ def main():
     start.record(stream)
     for i in range(K):
         ev[i][0].record(stream)
-        fa.fa_fwd(q, k, v, causal=W["causal"], out=o, lse=lse, stream=stream)
+        run_fwd(main_bufs, stream)
         ev[i][1].record(stream)
         if do_bwd:
-            fa.fa_bwd(q, k, v, o, lse, do, causal=W["causal"], dq=dq, dk=dk, dv=dv,
-                      workspace=ws, stream=stream)
+            run_bwd(main_bufs, stream)
         ev[i][2].record(stream)
     end.record(stream)
     barrier()
@@ -346,12 +382,9 @@ def main():
             stream.wait_event(in_done[b])
             if i >= 2:
                 stream.wait_event(out_done[b])  # step i-2's results have left these buffers
-            fa.fa_fwd(dbuf["q"], dbuf["k"], dbuf["v"], causal=W["causal"], out=dbuf["o"], lse=dbuf["lse"],
-                      stream=stream)
+            run_fwd(dbuf, stream)
             if do_bwd:
-                fa.fa_bwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["o"], dbuf["lse"], dbuf["do"],
-                          causal=W["causal"], dq=dbuf["dq"], dk=dbuf["dk"], dv=dbuf["dv"],
-                          workspace=dbuf["ws"], stream=stream)
+                run_bwd(dbuf, stream)
             comp_done[b].record(stream)
             s_out.wait_event(comp_done[b])
             with torch.cuda.stream(s_out):
