@@ -39,14 +39,14 @@ EncodeTiledFn encode_fn()
 // 4-D map over a [B, S, H, d] 16-bit tensor; one box = 64 head-dim columns x box_rows
 // rows of one (batch, head), 128-byte swizzled.  Rows past S read as zero.
 bool make_tmap(CUtensorMap* m, const void* ptr, int B, int S, int H, int d, bool bf16,
-               int box_rows = 128)
+               int box_rows = 128, int box_heads = 1)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
                                    (cuuint64_t)S * H * d * 2};
-    const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+    const cuuint32_t box[4] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
                const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -215,14 +215,19 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     st = device_info(&di);
     if (st != FA_OK) return st;
     const bool bf16 = dt == FA_BF16;
+    // Pack GQA: with few queries per head, the query heads that share a KV head fill the
+    // rows of a Q tile together (the group size must divide the 128-row tile)
+    const int group = Hq / Hkv;
+    const int pack = (group > 1 && group <= 16 && (group & (group - 1)) == 0 && Sq < 256) ? group : 1;
     CUtensorMap tq, tk, tv;
-    if (!make_tmap(&tq, q, B, Sq, Hq, d, bf16) || !make_tmap(&tk, k, B, Sk, Hkv, d, bf16) ||
+    if (!make_tmap(&tq, q, B, Sq, Hq, d, bf16, 128 / pack, pack) || !make_tmap(&tk, k, B, Sk, Hkv, d, bf16) ||
         !make_tmap(&tv, v, B, Sk, Hkv, d, bf16))
         return FA_ERR_CUDA;
     fa::FwdParams p{};
     p.o = o;
     p.lse = lse;
     p.Sq_alloc = Sq;
+    p.pack = pack;
     p.B = B;
     p.Sq = Sq;
     p.Sk = Sk;
@@ -230,9 +235,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     p.Hkv = Hkv;
     p.group = Hq / Hkv;
     const int unit = d == 128 ? 256 : 128;
-    p.num_m = (Sq + unit - 1) / unit;
-    p.num_tiles = B * Hq * p.num_m;
-    p.chunk_heads = chunk_heads_for(B, Hq, p.group, Sk, d);
+    p.num_m = (Sq * pack + unit - 1) / unit;
+    p.num_tiles = B * (pack > 1 ? Hkv : Hq) * p.num_m;
+    p.chunk_heads = pack > 1 ? chunk_heads_for(B, Hkv, 1, Sk, d) : chunk_heads_for(B, Hq, p.group, Sk, d);
     p.causal = causal ? 1 : 0;
     p.inject = take_inject();
     p.sl2 = scale * 1.4426950408889634f;
@@ -274,6 +279,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
     p.cu_k = cu_seqlens_k;
     p.used_k = seqused_k;
     p.Sq_alloc = total_q;
+    p.pack = 1;
     p.B = B;
     p.Sq = max_seqlen_q;
     p.Sk = max_seqlen_k;

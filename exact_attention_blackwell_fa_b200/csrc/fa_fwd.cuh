@@ -53,6 +53,10 @@ struct FwdParams {
     const int* cu_k;
     const int* used_k;
     int Sq_alloc;  // rows per batch entry of the q / o tensors (total_q when packed)
+    // pack > 1 ("pack GQA"): the `pack` (= group) query heads of a KV head share the
+    // rows of a Q tile, row r of a (batch, KV head) holding query r / pack of query
+    // head kv_head * pack + r % pack; units then run over (batch, KV head)
+    int pack;
     int B, Sq, Sk, Hq, Hkv, group;
     int num_m;        // query blocks per head
     int num_tiles;    // B * Hq * num_m
@@ -124,7 +128,8 @@ struct FwdCfg {
 template <int UNIT_ROWS>
 __device__ __forceinline__ void fwd_decode(const FwdParams& p, int t, int& b, int& h, int& m0)
 {
-    const int BH = p.B * p.Hq;
+    const int H = p.pack > 1 ? p.Hkv : p.Hq;  // heads of the unit list
+    const int BH = p.B * H;
     const int per_chunk = p.chunk_heads * p.num_m;
     const int c = t / per_chunk;
     const int r = t - c * per_chunk;
@@ -133,14 +138,16 @@ __device__ __forceinline__ void fwd_decode(const FwdParams& p, int t, int& b, in
     const int mi = r / csize;
     const int bh = first + (r - mi * csize);
     const int mblk = p.causal ? (p.num_m - 1 - mi) : mi;
-    b = bh / p.Hq;
-    h = bh - b * p.Hq;
+    b = bh / H;
+    h = bh - b * H;
     m0 = mblk * UNIT_ROWS;
 }
 
 // One work unit: UNIT_ROWS query rows of one (batch entry, query head).
 struct FwdUnit {
-    int b, h, m0;          // m0: first query row of the unit within its sequence
+    int b, h, m0;          // h: query head (KV head when packing); m0: first row of the
+                           // unit within its sequence's row space
+    int R;                 // rows of that space: Sq, or Sq * pack when packing
     int tb;                // batch coordinate in the TMA maps (0 for packed sequences)
     int q_base, k_base;    // tensor row of the sequence's first query / key
     int Sq, Sk;            // the sequence's query / key counts
@@ -168,13 +175,14 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int t)
         u.Sq = p.Sq;
         u.Sk = p.Sk;
     }
-    u.rows = u.m0 < u.Sq;
+    u.R = u.Sq * p.pack;
+    u.rows = u.m0 < u.R;
     // KV tiles to visit: all of the sequence's keys, or with the causal mask (key j
     // visible to query i iff j <= i + Sk - Sq) those up to the unit's last row's limit
     const int nk = (u.Sk + 127) / 128;
     u.n = u.rows ? nk : 0;
     if (u.rows && p.causal) {
-        const int last_row = min(u.m0 + UNIT_ROWS, u.Sq) - 1;
+        const int last_row = (min(u.m0 + UNIT_ROWS, u.R) - 1) / p.pack;
         const long long maxcol = static_cast<long long>(last_row) + u.Sk - u.Sq;
         u.n = maxcol < 0 ? 0 : min(nk, static_cast<int>(maxcol / 128) + 1);
     }
@@ -201,10 +209,12 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
         const FwdUnit u = fwd_unit<C::UNIT_ROWS>(p, t);
         if (!u.rows) continue;  // past the end of its (shorter) sequence: nothing to do
-        const int n = u.n, h = u.h;
-        const int q0 = u.m0 + q * C::BM;  // first query row of this Q tile
-        const int row = q0 + r_in_tile;
-        const bool row_ok = row < u.Sq;
+        const int n = u.n;
+        const int vr = u.m0 + q * C::BM + r_in_tile;  // this thread's row in the unit's row space
+        const int row = vr / p.pack;                  // its query
+        const int h = p.pack > 1 ? u.h * p.pack + (vr - row * p.pack) : u.h;
+        const int q0 = (u.m0 + q * C::BM) / p.pack;   // the Q tile's first (smallest) query
+        const bool row_ok = vr < u.R;
         const size_t orow_idx = static_cast<size_t>(u.tb) * p.Sq_alloc + u.q_base + row;
         T* orow = reinterpret_cast<T*>(p.o) + (orow_idx * p.Hq + h) * D;
         float* lrow = p.lse + (static_cast<size_t>(u.tb) * p.Hq + h) * p.Sq_alloc + u.q_base + row;
@@ -579,16 +589,19 @@ struct FwdLoad {
             const FwdUnit u = fwd_unit<C::UNIT_ROWS>(p, t);
             const int n = u.n, b = u.tb;
             if (n == 0) continue;
-            const int hkv = u.h / p.group;
+            const int hkv = p.pack > 1 ? u.h : u.h / p.group;
             // rows past the sequence's end (the next sequence's, or out of range) are
             // loaded too: their scores are masked, their outputs never stored
             auto krow = [&](int j) { return u.k_base + j * C::BN; };
             if (!wait_bar(bar(C::B_Q_EMPTY), (q_it & 1u) ^ 1u, ctl, W_FWD_Q_EMPTY)) return;
             mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_BYTES);
+            // packing: one box spans the group's `pack` heads x BM / pack queries, so
+            // shared-memory row r holds query r / pack of head r % pack
+            const int qh = p.pack > 1 ? u.h * p.pack : u.h;
             for (int q = 0; q < C::NQ; ++q)
                 for (int blk = 0; blk < D / 64; ++blk)
-                    tma_load_4d(sQ + q * C::QTILE + blk * 16384u, tmQ, bar(C::B_Q_FULL), blk * 64, u.h,
-                                u.q_base + u.m0 + q * C::BM, b);
+                    tma_load_4d(sQ + q * C::QTILE + blk * 16384u, tmQ, bar(C::B_Q_FULL), blk * 64, qh,
+                                u.q_base + (u.m0 + q * C::BM) / p.pack, b);
             q_round = static_cast<int>(q_it);
             ++q_it;
             if constexpr (C::NQ == 2) {
