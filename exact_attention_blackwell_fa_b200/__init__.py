@@ -5,6 +5,7 @@ device memory and the current stream; every step of the computation runs in the
 library's CUDA kernels.  The functions carry the C names:
 
     fa_fwd(q, k, v, causal=False, scale=None) -> (o, lse)
+    fa_fwd_splitkv(q, k, v, causal=False, scale=None, num_splits=0) -> (o, lse)
     fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
                   seqused_k=None, causal=False, scale=None) -> (o, lse)
     fa_bwd(q, k, v, o, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
@@ -31,7 +32,7 @@ import torch
 from . import _lib
 
 __all__ = [
-    "FAError", "fa_fwd", "fa_fwd_varlen", "fa_bwd", "fa_bwd_varlen", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
+    "FAError", "fa_fwd", "fa_fwd_splitkv", "fa_fwd_varlen", "fa_bwd", "fa_bwd_varlen", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
     "fa_last_device_status", "fa_clear_device_status", "fa_debug_inject", "fa_debug_exp2",
 ]
 
@@ -96,6 +97,33 @@ def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, 
                               lse.data_ptr(), B, Sq, Sk, Hq, Hkv, d, int(bool(causal)),
                               float(scale), _dtype_code(q), _stream_ptr(stream))
     _raise(code, "fa_fwd")
+    return out, lse
+
+
+def fa_fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, num_splits: int = 0,
+                   out=None, lse=None, workspace=None, stream=None):
+    """Split-KV forward (decode-shaped calls): same layouts and result as fa_fwd.
+    num_splits <= 0 lets the library choose."""
+    _check(q, "q")
+    _check(k, "k", q.dtype)
+    _check(v, "v", q.dtype)
+    B, Sq, Hq, d = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if k.shape != v.shape or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("fa: k and v must be [B, Sk, Hkv, d] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device=q.device)
+    lib = _lib.load()
+    if workspace is None:
+        need = int(lib.fa_fwd_splitkv_workspace_size(B, Sq, Sk, Hq, Hkv, d, int(num_splits)))
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    code = lib.fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq,
+                              Sk, Hq, Hkv, d, int(bool(causal)), float(scale), _dtype_code(q), int(num_splits),
+                              workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _raise(code, "fa_fwd_splitkv")
     return out, lse
 
 

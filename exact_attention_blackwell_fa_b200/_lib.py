@@ -20,6 +20,9 @@ _cf = ctypes.c_float
 _sz = ctypes.c_size_t
 SIGNATURES = {
     "fa_fwd": (_ci, [_vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp]),
+    "fa_fwd_splitkv_workspace_size": (_sz, [_ci, _ci, _ci, _ci, _ci, _ci, _ci]),
+    "fa_fwd_splitkv": (_ci, [_vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _ci, _ci, _vp,
+                             _sz, _vp]),
     "fa_fwd_varlen": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci,
                             _ci, _ci, _cf, _ci, _vp]),
     "fa_bwd_workspace_size": (_sz, [_ci, _ci, _ci, _ci]),

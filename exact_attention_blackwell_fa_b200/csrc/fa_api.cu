@@ -202,9 +202,10 @@ __global__ void fa_debug_exp2_kernel(const float* x, float* y, int n, int mode)
 
 extern "C" {
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
-                 int Sk, int Hq, int Hkv, int d, int causal, float scale, fa_dtype dt,
-                 fa_stream stream)
+// Dense forward; splits > 1 runs the split-KV form with partials in `workspace`.
+static fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
+                            int Sk, int Hq, int Hkv, int d, int causal, float scale, fa_dtype dt, int splits,
+                            void* workspace, fa_stream stream)
 {
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
     fa_status st = check_common(B, Sq, Sk, Hq, Hkv, d, scale, dt);
@@ -228,6 +229,13 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     p.lse = lse;
     p.Sq_alloc = Sq;
     p.pack = pack;
+    p.splits = splits;
+    if (splits > 1) {
+        const size_t part_rows = (size_t)splits * B * Hq * Sq;
+        p.opart = static_cast<float*>(workspace);
+        p.lsepart = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                             fa::bwd_round256(part_rows * d * 4));
+    }
     p.B = B;
     p.Sq = Sq;
     p.Sk = Sk;
@@ -236,17 +244,85 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     p.group = Hq / Hkv;
     const int unit = d == 128 ? 256 : 128;
     p.num_m = (Sq * pack + unit - 1) / unit;
-    p.num_tiles = B * (pack > 1 ? Hkv : Hq) * p.num_m;
+    p.num_tiles = B * (pack > 1 ? Hkv : Hq) * p.num_m * splits;
     p.chunk_heads = pack > 1 ? chunk_heads_for(B, Hkv, 1, Sk, d) : chunk_heads_for(B, Hq, p.group, Sk, d);
     p.causal = causal ? 1 : 0;
     p.inject = take_inject();
     p.sl2 = scale * 1.4426950408889634f;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (d == 128)
-        return bf16 ? launch_fwd<128, true>(tq, tk, tv, p, di.sm_count, s)
-                    : launch_fwd<128, false>(tq, tk, tv, p, di.sm_count, s);
-    return bf16 ? launch_fwd<256, true>(tq, tk, tv, p, di.sm_count, s)
-                : launch_fwd<256, false>(tq, tk, tv, p, di.sm_count, s);
+        st = bf16 ? launch_fwd<128, true>(tq, tk, tv, p, di.sm_count, s)
+                  : launch_fwd<128, false>(tq, tk, tv, p, di.sm_count, s);
+    else
+        st = bf16 ? launch_fwd<256, true>(tq, tk, tv, p, di.sm_count, s)
+                  : launch_fwd<256, false>(tq, tk, tv, p, di.sm_count, s);
+    if (st != FA_OK || splits == 1) return st;
+    const long long rows = (long long)B * Hq * Sq;
+    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    if (d == 128) {
+        if (bf16) fa::fa_fwd_combine_kernel<128, true><<<blocks, 256, 0, s>>>(p);
+        else fa::fa_fwd_combine_kernel<128, false><<<blocks, 256, 0, s>>>(p);
+    } else {
+        if (bf16) fa::fa_fwd_combine_kernel<256, true><<<blocks, 256, 0, s>>>(p);
+        else fa::fa_fwd_combine_kernel<256, false><<<blocks, 256, 0, s>>>(p);
+    }
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
+                 int Sk, int Hq, int Hkv, int d, int causal, float scale, fa_dtype dt,
+                 fa_stream stream)
+{
+    return fwd_common(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, d, causal, scale, dt, 1, nullptr, stream);
+}
+
+// Slices for the split-KV forward: enough units to cover the SMs, at least two KV
+// tiles per slice, at most 64 slices.
+static int splitkv_auto(int B, int Sq, int Sk, int Hq, int Hkv, int d, int sm_count)
+{
+    const int group = Hq / Hkv;
+    const int pack = (group > 1 && group <= 16 && (group & (group - 1)) == 0 && Sq < 256) ? group : 1;
+    const int unit = d == 128 ? 256 : 128;
+    const long long units = (long long)B * (pack > 1 ? Hkv : Hq) * ((Sq * pack + unit - 1) / unit);
+    const int nk = (Sk + 127) / 128;
+    long long s = (sm_count + units - 1) / units;
+    if (s > nk / 2) s = nk / 2;
+    if (s > 64) s = 64;
+    return s < 1 ? 1 : (int)s;
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int d, int num_splits)
+{
+    if (B < 1 || Sq < 1 || Sk < 1 || Hq < 1 || Hkv < 1 || (d != 128 && d != 256) || Hq % Hkv) return 0;
+    if (num_splits <= 0) {
+        DeviceInfo di;
+        if (device_info(&di) != FA_OK) return 0;
+        num_splits = splitkv_auto(B, Sq, Sk, Hq, Hkv, d, di.sm_count);
+    }
+    if (num_splits > 64) num_splits = 64;
+    const size_t rows = (size_t)num_splits * B * Hq * Sq;
+    return fa::bwd_round256(rows * d * 4) + fa::bwd_round256(rows * 4);
+}
+
+fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
+                         int Sk, int Hq, int Hkv, int d, int causal, float scale, fa_dtype dt, int num_splits,
+                         void* workspace, size_t workspace_bytes, fa_stream stream)
+{
+    if (num_splits > 64) return FA_ERR_INVALID_ARG;
+    if (num_splits <= 0) {
+        fa_status st = check_common(B, Sq, Sk, Hq, Hkv, d, scale, dt);
+        if (st != FA_OK) return st;
+        DeviceInfo di;
+        st = device_info(&di);
+        if (st != FA_OK) return st;
+        num_splits = splitkv_auto(B, Sq, Sk, Hq, Hkv, d, di.sm_count);
+    }
+    if (num_splits > 1) {
+        if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_INVALID_ARG;
+        if (workspace_bytes < fa_fwd_splitkv_workspace_size(B, Sq, Sk, Hq, Hkv, d, num_splits))
+            return FA_ERR_INVALID_ARG;
+    }
+    return fwd_common(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, d, causal, scale, dt, num_splits, workspace, stream);
 }
 
 fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -280,6 +356,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
     p.used_k = seqused_k;
     p.Sq_alloc = total_q;
     p.pack = 1;
+    p.splits = 1;
     p.B = B;
     p.Sq = max_seqlen_q;
     p.Sk = max_seqlen_k;

@@ -57,6 +57,13 @@ struct FwdParams {
     // rows of a Q tile, row r of a (batch, KV head) holding query r / pack of query
     // head kv_head * pack + r % pack; units then run over (batch, KV head)
     int pack;
+    // splits > 1 (split KV, for short query sequences over long key sequences): unit u
+    // covers the u-th of `splits` slices of the KV tiles and writes its O normalised by
+    // its own row sums to opart [splits][B][Hq][Sq][d] and its LSE (natural log, -inf
+    // for an empty slice) to lsepart [splits][B][Hq][Sq]; fa_fwd_combine_kernel merges
+    int splits;
+    float* opart;
+    float* lsepart;
     int B, Sq, Sk, Hq, Hkv, group;
     int num_m;        // query blocks per head
     int num_tiles;    // B * Hq * num_m
@@ -128,6 +135,7 @@ struct FwdCfg {
 template <int UNIT_ROWS>
 __device__ __forceinline__ void fwd_decode(const FwdParams& p, int t, int& b, int& h, int& m0)
 {
+    t /= p.splits;  // the slices of one unit are adjacent in the list
     const int H = p.pack > 1 ? p.Hkv : p.Hq;  // heads of the unit list
     const int BH = p.B * H;
     const int per_chunk = p.chunk_heads * p.num_m;
@@ -151,7 +159,9 @@ struct FwdUnit {
     int tb;                // batch coordinate in the TMA maps (0 for packed sequences)
     int q_base, k_base;    // tensor row of the sequence's first query / key
     int Sq, Sk;            // the sequence's query / key counts
-    int n;                 // KV tiles to visit
+    int n;                 // KV tiles to visit: j0 .. j0 + n - 1
+    int j0;                // first KV tile (split KV: the slice's first)
+    int split;             // slice index (split KV), else 0
     bool rows;             // the unit has query rows at all
 };
 
@@ -186,6 +196,13 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int t)
         const long long maxcol = static_cast<long long>(last_row) + u.Sk - u.Sq;
         u.n = maxcol < 0 ? 0 : min(nk, static_cast<int>(maxcol / 128) + 1);
     }
+    u.split = t % p.splits;
+    u.j0 = 0;
+    if (p.splits > 1) {
+        const int per = (u.n + p.splits - 1) / p.splits;
+        u.j0 = min(u.n, u.split * per);
+        u.n = min(u.n, u.j0 + per) - u.j0;
+    }
     return u;
 }
 
@@ -218,6 +235,17 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
         const size_t orow_idx = static_cast<size_t>(u.tb) * p.Sq_alloc + u.q_base + row;
         T* orow = reinterpret_cast<T*>(p.o) + (orow_idx * p.Hq + h) * D;
         float* lrow = p.lse + (static_cast<size_t>(u.tb) * p.Hq + h) * p.Sq_alloc + u.q_base + row;
+        // split KV: this slice's partial O and LSE rows
+        const size_t prow = ((static_cast<size_t>(u.split) * p.B + u.b) * p.Hq + h) * p.Sq + row;
+        if (n == 0 && p.splits > 1) {  // an empty slice
+            if (row_ok) {
+                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int c = 0; c < D / 4; ++c) reinterpret_cast<float4*>(p.opart + prow * D)[c] = z;
+                p.lsepart[prow] = -INFINITY;
+            }
+            continue;
+        }
         if (n == 0) {  // causal with Sq > Sk (or no keys): no key is visible to any row
             if (row_ok) {
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
@@ -255,7 +283,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
                 tmem_wait_ld_dep(a2);
                 tmem_wait_ld_dep(a3);
             }
-            const int c0 = j * C::BN;  // key index of column 0
+            const int c0 = (u.j0 + j) * C::BN;  // key index of column 0
             const bool masked = c0 + C::BN > lim0;
             if (masked) {
                 const int cut = lim - c0;
@@ -331,6 +359,24 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
         ++tile_it;
         tc_fence_after();
         const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
+        const float lse_row = (l > 0.0f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (p.splits > 1) {  // the slice's normalised O in fp32, and its LSE
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t r[32];
+                tmem_ld32_wait(tO + cc * 32, r);
+                if (row_ok) {
+                    float4* dst = reinterpret_cast<float4*>(p.opart + prow * D + cc * 32);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        dst[k] = make_float4(__uint_as_float(r[4 * k]) * inv, __uint_as_float(r[4 * k + 1]) * inv,
+                                             __uint_as_float(r[4 * k + 2]) * inv, __uint_as_float(r[4 * k + 3]) * inv);
+                }
+            }
+            if (row_ok) p.lsepart[prow] = lse_row;
+            tc_fence_before();
+            continue;
+        }
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t r[32];
@@ -347,7 +393,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
                 dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
             }
         }
-        if (row_ok) *lrow = (l > 0.0f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (row_ok) *lrow = lse_row;
         tc_fence_before();
     }
 }
@@ -592,7 +638,7 @@ struct FwdLoad {
             const int hkv = p.pack > 1 ? u.h : u.h / p.group;
             // rows past the sequence's end (the next sequence's, or out of range) are
             // loaded too: their scores are masked, their outputs never stored
-            auto krow = [&](int j) { return u.k_base + j * C::BN; };
+            auto krow = [&](int j) { return u.k_base + (u.j0 + j) * C::BN; };
             if (!wait_bar(bar(C::B_Q_EMPTY), (q_it & 1u) ^ 1u, ctl, W_FWD_Q_EMPTY)) return;
             mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_BYTES);
             // packing: one box spans the group's `pack` heads x BM / pack queries, so
@@ -710,6 +756,58 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == C::CTRL_WARP) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------------
+// Split KV: merge the slices.  One warp per (b, h, query row): LSE = log sum_p e^LSE_p,
+// O = sum_p e^(LSE_p - LSE) O_p (each O_p normalised by its own slice's row sum).
+// ---------------------------------------------------------------------------------
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_fwd_combine_kernel(const FwdParams p)
+{
+    const int lane = threadIdx.x & 31;
+    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const long long rows = static_cast<long long>(p.B) * p.Hq * p.Sq;  // (b, h, i)
+    if (row >= rows) return;
+    const int i = static_cast<int>(row % p.Sq);
+    const long long bh = row / p.Sq;
+    const int h = static_cast<int>(bh % p.Hq), b = static_cast<int>(bh / p.Hq);
+    float m = -INFINITY;
+    for (int s = 0; s < p.splits; ++s) m = fmaxf(m, p.lsepart[static_cast<size_t>(s) * rows + row]);
+    constexpr int PER = D / 32;  // values per lane
+    float acc[PER];
+#pragma unroll
+    for (int c = 0; c < PER; ++c) acc[c] = 0.0f;
+    float sum = 0.0f;
+    if (m != -INFINITY) {
+        for (int s = 0; s < p.splits; ++s) {
+            const float ls = p.lsepart[static_cast<size_t>(s) * rows + row];
+            if (ls == -INFINITY) continue;
+            const float w = expf(ls - m);
+            sum += w;
+            const float* src = p.opart + (static_cast<size_t>(s) * rows + row) * D + lane * PER;
+#pragma unroll
+            for (int c = 0; c < PER; c += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(src + c);
+                acc[c] = fmaf(w, x.x, acc[c]);
+                acc[c + 1] = fmaf(w, x.y, acc[c + 1]);
+                acc[c + 2] = fmaf(w, x.z, acc[c + 2]);
+                acc[c + 3] = fmaf(w, x.w, acc[c + 3]);
+            }
+        }
+    }
+    const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+    uint16_t* dst = static_cast<uint16_t*>(p.o) + ((static_cast<size_t>(b) * p.Sq + i) * p.Hq + h) * D + lane * PER;
+    uint32_t w[PER / 2];
+#pragma unroll
+    for (int c = 0; c < PER / 2; ++c) w[c] = pack2<BF16>(acc[2 * c] * inv, acc[2 * c + 1] * inv);
+    if constexpr (PER == 4) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+    } else {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (lane == 0)
+        p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Sq + i] = m == -INFINITY ? -INFINITY : m + logf(sum);
 }
 
 }  // namespace fa

@@ -67,6 +67,22 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  fa_dtype dt, fa_stream stream);
 
 /*
+ * Split-KV forward, for short query sequences over long key sequences (decode):
+ * the same result as fa_fwd, with the key range of every (batch, head, query
+ * block) cut into num_splits slices processed by separate CTAs, so that few query
+ * rows still occupy the whole GPU; a second kernel merges the slices
+ * (LSE = log sum_p e^LSE_p, O = sum_p e^(LSE_p - LSE) O_p).  num_splits <= 0 picks
+ * a count from the shape and the SM count; at most 64.  With more than one slice
+ * the caller provides `workspace` (256-byte aligned, at least
+ * fa_fwd_splitkv_workspace_size(...) bytes, same num_splits) for the slices'
+ * float32 partial O and LSE.  Layouts, dtypes and errors as fa_fwd.
+ */
+size_t fa_fwd_splitkv_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int d, int num_splits);
+fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
+                         int Sk, int Hq, int Hkv, int d, int causal, float scale, fa_dtype dt, int num_splits,
+                         void* workspace, size_t workspace_bytes, fa_stream stream);
+
+/*
  * Forward over a packed batch of variable-length sequences (the varlen row of
  * "[RFC] FA4 -- head_dim=256 & head_dim=512", Phase 1: cu_seqlens and seqused_k).
  * Sequence b's queries are rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 of
