@@ -183,6 +183,11 @@ def main():
     ap.add_argument("--hd", type=int, default=None)
     ap.add_argument("--causal", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--q-len", type=int, default=None,
+                    help="query rows per sequence (default: --seq); a short one over long keys is "
+                         "decode-shaped")
+    ap.add_argument("--splitkv", action="store_true",
+                    help="forward through fa_fwd_splitkv (slice count chosen by the library)")
     ap.add_argument("--varlen", default=None,
                     help="comma-separated sequence lengths: one packed batch of these sequences "
                          "(fa_fwd_varlen / fa_bwd_varlen) instead of the dense workload")
@@ -203,7 +208,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     W = WORKLOAD
+    W["Sq"] = args.q_len if args.q_len is not None else W["S"]
     lens = [int(x) for x in args.varlen.split(",")] if args.varlen else None
+    if lens and (args.q_len is not None or args.splitkv):
+        raise SystemExit("--varlen does not combine with --q-len / --splitkv")
     if lens:
         W["B"], W["S"] = len(lens), max(lens)
         f_fwd = sum(flops(1, L, L, W["H"], W["d"], W["causal"])[0] for L in lens)
@@ -211,16 +219,18 @@ def main():
         wl = (f"attention fwd+bwd bf16 varlen packed lens={','.join(map(str, lens))} H={W['H']} "
               f"Hkv={W['Hkv']} d={W['d']} {'causal' if W['causal'] else 'non-causal'}")
     else:
-        f_fwd, f_bwd = flops(W["B"], W["S"], W["S"], W["H"], W["d"], W["causal"])
-        wl = (f"attention fwd+bwd bf16 B={W['B']} S={W['S']} H={W['H']} Hkv={W['Hkv']} d={W['d']} "
-              f"{'causal' if W['causal'] else 'non-causal'}")
+        f_fwd, f_bwd = flops(W["B"], W["Sq"], W["S"], W["H"], W["d"], W["causal"])
+        sq = "" if W["Sq"] == W["S"] else f" Sq={W['Sq']}"
+        wl = (f"attention fwd+bwd bf16 B={W['B']} S={W['S']}{sq} H={W['H']} Hkv={W['Hkv']} d={W['d']} "
+              f"{'causal' if W['causal'] else 'non-causal'}" + (" split-KV" if args.splitkv else ""))
     config = {"workload": wl,
               "B": W["B"], "seq_len": W["S"], "heads": W["H"], "kv_heads": W["Hkv"],
               "head_dim": W["d"],
               "causal": W["causal"], "global_batch": W["B"] * world,
               "parallelism": f"replicas x{world} (independent batches, no collective)",
-              "l2": ("inputs larger than L2 (each of Q, O, dO is "
-                     f"{(sum(lens) if lens else W['B'] * W['S']) * W['H'] * W['d'] * 2 / 2**20:.0f} MiB)")}
+              "l2": (f"Q, O, dO {(sum(lens) if lens else W['B'] * W['Sq']) * W['H'] * W['d'] * 2 / 2**20:.0f} MiB "
+                     f"each, K, V {(sum(lens) if lens else W['B'] * W['S']) * W['Hkv'] * W['d'] * 2 / 2**20:.0f} "
+                     "MiB each (L2: 126 MB)")}
     if lens:
         config["seq_lens"] = lens
 
@@ -265,13 +275,19 @@ def main():
         cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0)), dtype=torch.int32, device=dev)
         lse = torch.empty(W["H"], total, dtype=torch.float32, device=dev)
     else:
-        shape = Shape(W["B"], W["S"], W["S"], W["H"], W["Hkv"], W["d"])
+        shape = Shape(W["B"], W["Sq"], W["S"], W["H"], W["Hkv"], W["d"])
         q, k, v, do = make_inputs(shape, seed=rank, device=dev, with_dout=True)
-        lse = torch.empty(W["B"], W["H"], W["S"], dtype=torch.float32, device=dev)
+        lse = torch.empty(W["B"], W["H"], W["Sq"], dtype=torch.float32, device=dev)
     o = torch.empty_like(q)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(fa.fa_bwd_workspace_size(W["B"], W["S"], W["H"], W["d"]), dtype=torch.uint8,
+    ws = torch.empty(fa.fa_bwd_workspace_size(W["B"], W["Sq"], W["H"], W["d"]), dtype=torch.uint8,
                      device=dev)
+    split_ws = None
+    if args.splitkv:
+        from exact_attention_blackwell_fa_b200 import _lib as _fal
+        need = int(_fal.load().fa_fwd_splitkv_workspace_size(W["B"], W["Sq"], W["S"], W["H"], W["Hkv"],
+                                                             W["d"], 0))
+        split_ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     main_bufs = dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws)
 
@@ -280,6 +296,9 @@ def main():
         if lens:
             fa.fa_fwd_varlen(t["q"], t["k"], t["v"], cu, cu, W["S"], W["S"], causal=W["causal"], out=t["o"],
                              lse=t["lse"], stream=st)
+        elif args.splitkv:
+            fa.fa_fwd_splitkv(t["q"], t["k"], t["v"], causal=W["causal"], out=t["o"], lse=t["lse"],
+                              workspace=split_ws, stream=st)
         else:
             fa.fa_fwd(t["q"], t["k"], t["v"], causal=W["causal"], out=t["o"], lse=t["lse"], stream=st)
 
@@ -408,6 +427,17 @@ def main():
         dom, dom_ms, dom_flops = "fa_fwd_kernel", fwd_ms, f_fwd
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+            "peak_kind": f"{peak_kind} sustained bf16 (cuBLAS loop)", "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": recorded_traffic(dom, config["workload"])}
+    if args.splitkv and not do_bwd:
+        # decode-shaped: bound by reading K and V (plus Q, O, LSE) once from HBM
+        alg = nbytes(q, k, v, o, lse)
+        gbs = alg / (fwd_ms * 1e-3) / 1e9
+        hpeak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        roof = {"bound": "hbm", "kernel": "fa_fwd_splitkv (slices + combine)", "achieved": gbs, "peak": hpeak,
+                "peak_kind": f"{peak_kind} HBM copy", "unit": "GB/s", "frac": gbs / hpeak,
+                "algorithmic_bytes": alg, "traffic": None}
     out = {
         "metric": "attention fwd/bwd TFLOPS at 1 B200 and fraction of 2.25 PFLOPS BF16 peak",
         "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -420,10 +450,7 @@ def main():
         "bwd": ({"ms": bwd_ms, "tflops": f_bwd / (bwd_ms * 1e-3) / 1e12,
                  "frac_of_2250": f_bwd / (bwd_ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS}
                 if do_bwd else None),
-        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
-                     "peak_kind": f"{peak_kind} sustained bf16 (cuBLAS loop)",
-                     "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": recorded_traffic(dom, config["workload"])},
+        "roofline": roof,
         "e2e": e2e,
         "gpu_launches": K * (1 + (3 if do_bwd else 0)),
         "clocks": clocks,
