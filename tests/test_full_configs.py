@@ -124,3 +124,89 @@ def test_full_bwd_d128(oracle_mod, S, causal):
 
 def test_full_bwd_d256(oracle_mod):
     _check_bwd(oracle_mod, Shape(1, 16384, 16384, 8, 8, 256), False)
+
+
+# ---- the widened rows at full size -------------------------------------------------
+
+def _sampled_rows_check(oracle_mod, q, k, v, o, lse, causal, rows):
+    """O and LSE of the given (b, h, i) rows against the oracle."""
+    o_ref, lse_ref = oracle_mod.fwd(q, k, v, causal=causal, rows=rows)
+    b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+    got = o[b.cuda(), i.cuda(), h.cuda()].cpu().double()
+    err = (got - o_ref).abs()
+    assert (err - (O_MAX + _half_ulp(o_ref))).max().item() <= 0.0, err.max().item()
+    assert err.mean().item() <= O_MEAN
+    gl = lse[b.cuda(), h.cuda(), i.cuda()].cpu().double()
+    fin = torch.isfinite(lse_ref)
+    assert torch.equal(torch.isfinite(gl), fin)
+    if fin.any():
+        assert (gl[fin] - lse_ref[fin]).abs().max().item() <= LSE_MAX
+
+
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_splitkv_decode_long_keys(oracle_mod, causal, d):
+    """Decode over 128k keys: 4 sequences x 1 (and 8) queries, 32 / 4 heads."""
+    import exact_attention_blackwell_fa_b200 as fa
+
+    for Sq in (1, 8):
+        shape = Shape(4, Sq, 131072, 32 if d == 128 else 16, 4 if d == 128 else 2, d)
+        q, k, v = make_inputs(shape, seed=Sq)
+        o, lse = fa.fa_fwd_splitkv(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+        torch.cuda.synchronize()
+        assert fa.fa_last_device_status()[0] == 0
+        rows = sample_rows(shape.B, shape.Hq, Sq, Sq, seed=3)
+        _sampled_rows_check(oracle_mod, q, k, v, o, lse, causal, rows)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_pack_gqa_chunk(oracle_mod, causal):
+    """A 64-query chunk against 32k keys per sequence, group of 8 (pack GQA)."""
+    import exact_attention_blackwell_fa_b200 as fa
+
+    shape = Shape(8, 64, 32768, 32, 4, 128)
+    q, k, v = make_inputs(shape, seed=5)
+    o, lse = fa.fa_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    torch.cuda.synchronize()
+    rows = sample_rows(shape.B, shape.Hq, shape.Sq, 2, seed=4)
+    _sampled_rows_check(oracle_mod, q, k, v, o, lse, causal, rows)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_varlen_packed_32k_tokens(oracle_mod, causal):
+    """One packed batch of 32,640 tokens (lengths 16384 .. 128), H=16, d=128: forward
+    rows sampled from every sequence, and the backward's dQ on sampled rows and dK/dV
+    on sampled keys of the longest and shortest sequences."""
+    import exact_attention_blackwell_fa_b200 as fa
+
+    lens = [16384, 8192, 4096, 2048, 1024, 512, 256, 128]
+    H, d = 16, 128
+    tot = sum(lens)
+    q, k, v, do = (t[0] for t in make_inputs(Shape(1, tot, tot, H, H, d), seed=11, with_dout=True))
+    cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0)), dtype=torch.int32)
+    qc, kc, vc, doc, cuc = q.cuda(), k.cuda(), v.cuda(), do.cuda(), cu.cuda()
+    o, lse = fa.fa_fwd_varlen(qc, kc, vc, cuc, cuc, max(lens), max(lens), causal=causal)
+    dq, dk, dv = fa.fa_bwd_varlen(qc, kc, vc, o, lse, doc, cuc, cuc, max(lens), max(lens), causal=causal)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status()[0] == 0
+    for s, L in enumerate(lens):
+        a = int(cu[s])
+        qs, ks, vs, dos = (t[a:a + L].unsqueeze(0) for t in (q, k, v, do))
+        rows = sample_rows(1, H, L, 2, seed=s)
+        b_, h_, i_ = rows[:, 0], rows[:, 1], rows[:, 2]
+        o_ref, lse_ref = oracle_mod.fwd(qs, ks, vs, causal=causal, rows=rows)
+        got = o[(a + i_).cuda(), h_.cuda()].cpu().double()
+        err = (got - o_ref).abs()
+        assert (err - (O_MAX + _half_ulp(o_ref))).max().item() <= 0.0, (L, err.max().item())
+        gl = lse[h_.cuda(), (a + i_).cuda()].cpu().double()
+        assert (gl - lse_ref).abs().max().item() <= LSE_MAX
+        if s in (0, len(lens) - 1):
+            qrows = sample_rows(1, H, L, 1, seed=s + 100)
+            js = torch.unique(torch.tensor([0, L - 1, L // 2]))
+            kvrows = torch.stack([torch.zeros_like(js), torch.full_like(js, H - 1), js], 1)
+            rq, rk, rv, _ = oracle_mod.bwd(qs, ks, vs, dos, causal=causal, qrows=qrows, kvrows=kvrows)
+            gq = dq[(a + qrows[:, 2]).cuda(), qrows[:, 1].cuda()].cpu().double()
+            gk = dk[(a + js).cuda(), H - 1].cpu().double()
+            gv = dv[(a + js).cuda(), H - 1].cpu().double()
+            for name, g_, r_ in (("dq", gq, rq), ("dk", gk, rk), ("dv", gv, rv)):
+                assert (g_ - r_).abs().max().item() <= GRAD_REL * r_.abs().max().item(), (L, name)
