@@ -11,7 +11,7 @@ LIB = os.path.join(HERE, "libfa.so")
 ROOT = os.path.dirname(HERE)
 
 SOURCES = ["fa_api.cu"]
-DEPS = ["fa_api.cu", "fa_fwd.cuh", "fa_bwd.cuh", "fa_bwd256.cuh", "fa_common.cuh", "sm100.cuh", "exp2_poly.h"]
+DEPS = ["fa_api.cu", "fa_fwd.cuh", "fa_bwd.cuh", "fa_bwd_wide.cuh", "fa_common.cuh", "sm100.cuh", "exp2_poly.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

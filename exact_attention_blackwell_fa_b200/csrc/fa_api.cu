@@ -11,7 +11,7 @@
 
 #include "../../include/fa.h"
 #include "fa_bwd.cuh"
-#include "fa_bwd256.cuh"
+#include "fa_bwd_wide.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -88,7 +88,7 @@ fa_status check_common(int B, int Sq, int Sk, int Hq, int Hkv, int d, float scal
     if (B < 1 || Sq < 1 || Sk < 1 || Hq < 1 || Hkv < 1) return FA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
-    if (d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+    if (d != 128 && d != 192 && d != 256) return FA_ERR_UNSUPPORTED;
     if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_UNSUPPORTED;
     // element counts must stay inside the 32-bit row indices the kernels use
     const long long rows_q = (long long)B * Sq * Hq, rows_k = (long long)B * Sk * Hkv;
@@ -146,22 +146,22 @@ fa_status launch_bwd_d128(const CUtensorMap& tq, const CUtensorMap& tk, const CU
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <bool BF16>
-fa_status launch_bwd_d256(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64,
+template <int D, bool BF16>
+fa_status launch_bwd_wide(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64,
                           const CUtensorMap& tdo, const fa::BwdParams& p, int sm_count,
                           cudaStream_t stream)
 {
-    using C = fa::Bwd256Cfg<BF16>;
+    using C = fa::BwdWideCfg<D, BF16>;
     const long long pre_rows = (long long)p.B * p.Hq * p.Sq_pad;
-    fa::fa_bwd_pre_kernel<256, BF16><<<(unsigned)((pre_rows + 7) / 8), 256, 0, stream>>>(p);
+    fa::fa_bwd_pre_kernel<D, BF16><<<(unsigned)((pre_rows + 7) / 8), 256, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    fa_status st = set_smem(fa::fa_bwd_dkdv256_kernel<BF16>, C::SMEM_BYTES);
+    fa_status st = set_smem(fa::fa_bwd_dkdv_wide_kernel<D, BF16>, C::SMEM_BYTES);
     if (st != FA_OK) return st;
     const int grid = p.num_units < sm_count ? p.num_units : sm_count;
-    fa::fa_bwd_dkdv256_kernel<BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk64, tv64, tdo, p);
+    fa::fa_bwd_dkdv_wide_kernel<D, BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk64, tv64, tdo, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     const long long dq_rows = (long long)p.B * p.Sq * p.Hq;
-    fa::fa_bwd_dq_kernel<256, BF16><<<(unsigned)((dq_rows + 7) / 8), 256, 0, stream>>>(p);
+    fa::fa_bwd_dq_kernel<D, BF16><<<(unsigned)((dq_rows + 7) / 8), 256, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -176,6 +176,27 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
     const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
     fa::fa_fwd_kernel<D, BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// query rows per forward work unit: two 128-row Q tiles at head_dim 128, one otherwise
+int fwd_unit_rows(int d) { return d == 128 ? 256 : 128; }
+
+fa_status launch_fwd_any(int d, bool bf16, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const fa::FwdParams& p, int sm_count, cudaStream_t s)
+{
+    switch (d) {
+    case 128: return bf16 ? launch_fwd<128, true>(tq, tk, tv, p, sm_count, s) : launch_fwd<128, false>(tq, tk, tv, p, sm_count, s);
+    case 192: return bf16 ? launch_fwd<192, true>(tq, tk, tv, p, sm_count, s) : launch_fwd<192, false>(tq, tk, tv, p, sm_count, s);
+    case 256: return bf16 ? launch_fwd<256, true>(tq, tk, tv, p, sm_count, s) : launch_fwd<256, false>(tq, tk, tv, p, sm_count, s);
+    default: return FA_ERR_UNSUPPORTED;
+    }
+}
+
+template <int D>
+void launch_combine(bool bf16, const fa::FwdParams& p, unsigned blocks, cudaStream_t s)
+{
+    if (bf16) fa::fa_fwd_combine_kernel<D, true><<<blocks, 256, 0, s>>>(p);
+    else fa::fa_fwd_combine_kernel<D, false><<<blocks, 256, 0, s>>>(p);
 }
 
 }  // namespace
@@ -242,7 +263,7 @@ static fa_status fwd_common(const void* q, const void* k, const void* v, void* o
     p.Hq = Hq;
     p.Hkv = Hkv;
     p.group = Hq / Hkv;
-    const int unit = d == 128 ? 256 : 128;
+    const int unit = fwd_unit_rows(d);
     p.num_m = (Sq * pack + unit - 1) / unit;
     p.num_tiles = B * (pack > 1 ? Hkv : Hq) * p.num_m * splits;
     p.chunk_heads = pack > 1 ? chunk_heads_for(B, Hkv, 1, Sk, d) : chunk_heads_for(B, Hq, p.group, Sk, d);
@@ -250,22 +271,13 @@ static fa_status fwd_common(const void* q, const void* k, const void* v, void* o
     p.inject = take_inject();
     p.sl2 = scale * 1.4426950408889634f;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (d == 128)
-        st = bf16 ? launch_fwd<128, true>(tq, tk, tv, p, di.sm_count, s)
-                  : launch_fwd<128, false>(tq, tk, tv, p, di.sm_count, s);
-    else
-        st = bf16 ? launch_fwd<256, true>(tq, tk, tv, p, di.sm_count, s)
-                  : launch_fwd<256, false>(tq, tk, tv, p, di.sm_count, s);
+    st = launch_fwd_any(d, bf16, tq, tk, tv, p, di.sm_count, s);
     if (st != FA_OK || splits == 1) return st;
     const long long rows = (long long)B * Hq * Sq;
     const unsigned blocks = (unsigned)((rows + 7) / 8);
-    if (d == 128) {
-        if (bf16) fa::fa_fwd_combine_kernel<128, true><<<blocks, 256, 0, s>>>(p);
-        else fa::fa_fwd_combine_kernel<128, false><<<blocks, 256, 0, s>>>(p);
-    } else {
-        if (bf16) fa::fa_fwd_combine_kernel<256, true><<<blocks, 256, 0, s>>>(p);
-        else fa::fa_fwd_combine_kernel<256, false><<<blocks, 256, 0, s>>>(p);
-    }
+    if (d == 128) launch_combine<128>(bf16, p, blocks, s);
+    else if (d == 192) launch_combine<192>(bf16, p, blocks, s);
+    else launch_combine<256>(bf16, p, blocks, s);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -282,7 +294,7 @@ static int splitkv_auto(int B, int Sq, int Sk, int Hq, int Hkv, int d, int sm_co
 {
     const int group = Hq / Hkv;
     const int pack = (group > 1 && group <= 16 && (group & (group - 1)) == 0 && Sq < 256) ? group : 1;
-    const int unit = d == 128 ? 256 : 128;
+    const int unit = fwd_unit_rows(d);
     const long long units = (long long)B * (pack > 1 ? Hkv : Hq) * ((Sq * pack + unit - 1) / unit);
     const int nk = (Sk + 127) / 128;
     long long s = (sm_count + units - 1) / units;
@@ -293,7 +305,7 @@ static int splitkv_auto(int B, int Sq, int Sk, int Hq, int Hkv, int d, int sm_co
 
 size_t fa_fwd_splitkv_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int d, int num_splits)
 {
-    if (B < 1 || Sq < 1 || Sk < 1 || Hq < 1 || Hkv < 1 || (d != 128 && d != 256) || Hq % Hkv) return 0;
+    if (B < 1 || Sq < 1 || Sk < 1 || Hq < 1 || Hkv < 1 || (d != 128 && d != 192 && d != 256) || Hq % Hkv) return 0;
     if (num_splits <= 0) {
         DeviceInfo di;
         if (device_info(&di) != FA_OK) return 0;
@@ -363,19 +375,14 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
     p.Hq = Hq;
     p.Hkv = Hkv;
     p.group = Hq / Hkv;
-    const int unit = d == 128 ? 256 : 128;
+    const int unit = fwd_unit_rows(d);
     p.num_m = (max_seqlen_q + unit - 1) / unit;
     p.num_tiles = B * Hq * p.num_m;
     p.chunk_heads = chunk_heads_for(B, Hq, p.group, max_seqlen_k, d);
     p.causal = causal ? 1 : 0;
     p.inject = take_inject();
     p.sl2 = scale * 1.4426950408889634f;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (d == 128)
-        return bf16 ? launch_fwd<128, true>(tq, tk, tv, p, di.sm_count, s)
-                    : launch_fwd<128, false>(tq, tk, tv, p, di.sm_count, s);
-    return bf16 ? launch_fwd<256, true>(tq, tk, tv, p, di.sm_count, s)
-                : launch_fwd<256, false>(tq, tk, tv, p, di.sm_count, s);
+    return launch_fwd_any(d, bf16, tq, tk, tv, p, di.sm_count, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int Sq, int Hq, int d)
@@ -452,8 +459,11 @@ static fa_status bwd_common(const void* q, const void* k, const void* v, const v
     p.sl2 = scale * 1.4426950408889634f;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (d == 256)
-        return bf16 ? launch_bwd_d256<true>(tq, tk, tv, tdo, p, di.sm_count, s)
-                    : launch_bwd_d256<false>(tq, tk, tv, tdo, p, di.sm_count, s);
+        return bf16 ? launch_bwd_wide<256, true>(tq, tk, tv, tdo, p, di.sm_count, s)
+                    : launch_bwd_wide<256, false>(tq, tk, tv, tdo, p, di.sm_count, s);
+    if (d == 192)
+        return bf16 ? launch_bwd_wide<192, true>(tq, tk, tv, tdo, p, di.sm_count, s)
+                    : launch_bwd_wide<192, false>(tq, tk, tv, tdo, p, di.sm_count, s);
     return bf16 ? launch_bwd_d128<true>(tq, tk, tv, tdo, p, di.sm_count, s)
                 : launch_bwd_d128<false>(tq, tk, tv, tdo, p, di.sm_count, s);
 }

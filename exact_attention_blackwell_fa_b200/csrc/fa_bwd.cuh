@@ -122,7 +122,13 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p)
         const size_t off = (trow * p.Hq + h) * D + lane * (D / 32);
         constexpr int NW = D / 64;  // 32-bit words per lane (two 16-bit values each)
         uint32_t ow[NW], dw[NW];
-        if constexpr (NW == 2) {
+        if constexpr (NW == 3) {  // 12 bytes per lane: 4-byte aligned only
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                ow[w] = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.o) + off)[w];
+                dw[w] = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.dout) + off)[w];
+            }
+        } else if constexpr (NW == 2) {
             const uint2 a = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.o) + off);
             const uint2 c = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.dout) + off);
             ow[0] = a.x; ow[1] = a.y; dw[0] = c.x; dw[1] = c.y;
@@ -175,7 +181,13 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p)
     const size_t trow = static_cast<size_t>(sq.tb) * p.Sq_alloc + sq.q_base + i;
     const float* src = p.dqacc + ((static_cast<size_t>(b) * p.Hq + h) * p.Sq_pad + i) * D + lane * (D / 32);
     uint16_t* dst = static_cast<uint16_t*>(p.dq) + (trow * p.Hq + h) * D + lane * (D / 32);
-    if constexpr (D == 128) {
+    if constexpr (D == 192) {  // 6 values per lane: 8-byte loads, 4-byte stores
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+            const float2 a = reinterpret_cast<const float2*>(src)[c];
+            reinterpret_cast<uint32_t*>(dst)[c] = pack2<BF16>(a.x * p.scale, a.y * p.scale);
+        }
+    } else if constexpr (D == 128) {
         const float4 a = *reinterpret_cast<const float4*>(src);
         *reinterpret_cast<uint2*>(dst) =
             make_uint2(pack2<BF16>(a.x * p.scale, a.y * p.scale), pack2<BF16>(a.z * p.scale, a.w * p.scale));

@@ -1,4 +1,5 @@
-// fa_bwd256.cuh -- dK / dV / dQ-partials kernel of the attention backward for head_dim 256.
+// fa_bwd_wide.cuh -- dK / dV / dQ-partials kernel of the attention backward for head_dim
+// 192 and 256.
 //
 // Same arithmetic as the head_dim 128 kernel in fa_bwd.cuh (P recomputed from LSE,
 // dS = P (dP - D), dV = P^T dO, dK = scale dS^T Q, dQ partials reduced in fp32), with
@@ -17,6 +18,11 @@
 //     region (head dims on the lanes), each drained by the dQ warpgroup into the fp32
 //     accumulator, one 128-byte segment per warp-wide reduction.
 //
+// head_dim 192 runs the same tiling with the fourth 64-dim block of every operand tile
+// zero: it is cleared once, TMA never writes it, the d-contractions (S, dP) stop at
+// dim 192, and the second head-dim half of dV^T, dK^T and dQ^T has 64 live lanes (the
+// other 64 are zero and never read).
+//
 // TMEM: S [0,64) | dP [64,128) | dQ^T half [128,256) | dV^T halves [256,384) | dK^T [384,512)
 #pragma once
 
@@ -24,9 +30,11 @@
 
 namespace fa {
 
-template <bool BF16>
-struct Bwd256Cfg {
-    static constexpr int D = 256;
+template <int DIM, bool BF16>
+struct BwdWideCfg {
+    static_assert(DIM == 192 || DIM == 256, "head_dim");
+    static constexpr int D = DIM;
+    static constexpr int NB = D / 64;  // 64-dim blocks loaded per operand tile
     static constexpr int BN = 64;   // keys per unit
     static constexpr int BM = 128;  // query rows per step
     // warps 0-7: compute (two warpgroups, 32 keys each), 8-11: dQ, 12: MMA, 13: TMA,
@@ -35,16 +43,17 @@ struct Bwd256Cfg {
     static constexpr int DQ_WARP = 8, MMA_WARP = 12, LOAD_WARP = 13;
     // registers per thread: launched at 128; the MMA/TMA warpgroup gives 8 of them to
     // the dQ warpgroup, which then holds a whole 128-column dQ^T row in registers
-    static constexpr uint32_t REG_LAUNCH = 128, REG_DQ = 136, REG_CTRL = 120;
+    static constexpr uint32_t REG_LAUNCH = 128, REG_DQ = D == 256 ? 136 : 144, REG_CTRL = D == 256 ? 120 : 112;
     static_assert(8 * 32 * REG_LAUNCH + 4 * 32 * REG_DQ + 4 * 32 * REG_CTRL <= THREADS * REG_LAUNCH,
                   "register split exceeds the launch budget");
     // lane 0 of the MMA warp issues alone (the converged, elected-lane form measured
     // slower here)
     static constexpr bool WARP_ISSUE = false;
     static constexpr uint32_t KV_BLK = BN * 128;   // [64 rows][64 cols] of 16-bit values
-    static constexpr uint32_t KV_BYTES = 4 * KV_BLK;
+    static constexpr uint32_t KV_BYTES = 4 * KV_BLK;  // space: four blocks
     static constexpr uint32_t Q_BLK = BM * 128;    // [128 rows][64 cols]
     static constexpr uint32_t Q_BYTES = 4 * Q_BLK;
+    static constexpr uint32_t KV_LOAD = NB * KV_BLK, Q_LOAD = NB * Q_BLK;  // bytes copied
     static constexpr uint32_t PT_BYTES = BM * BN * 2;  // [128 queries][64 keys]
     static constexpr uint32_t ROWS_BYTES = 1024;       // LSE*log2(e)[128], D[128]
     static constexpr uint32_t OFF_K = 0, OFF_V = KV_BYTES, OFF_Q = 2 * KV_BYTES,
@@ -72,7 +81,7 @@ enum : uint32_t {
 };
 
 // num_n counts 64-key blocks here
-__device__ __forceinline__ BwdUnit bwd256_decode(const BwdParams& p, int t)
+__device__ __forceinline__ BwdUnit bwd_wide_decode(const BwdParams& p, int t)
 {
     const int BH = p.B * p.Hkv;
     const int per_chunk = p.chunk_heads * p.num_n;
@@ -121,11 +130,11 @@ __device__ __forceinline__ void store_tile_half_row(uint32_t tile, int row, int 
 }
 
 // ---- compute warpgroups (thread = query row, 32 keys each): P and dS; epilogue ----
-template <bool BF16>
-__device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars,
+template <int D, bool BF16>
+__device__ void bwd_wide_compute(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars,
                                CtaCtl* ctl, int wq, int half)
 {
-    using C = Bwd256Cfg<BF16>;
+    using C = BwdWideCfg<D, BF16>;
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
     const int lane = threadIdx.x & 31;
     const int t = wq * 32 + lane;  // query row within the block, and head-dim lane later
@@ -135,7 +144,7 @@ __device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base,
     const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
     uint32_t it = 0, unit_it = 0;
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
-        const BwdUnit u = bwd256_decode(p, ui);
+        const BwdUnit u = bwd_wide_decode(p, ui);
         if (!u.keys) continue;  // past the end of its sequence's keys
         // dV^T / dK^T element of head-dim column (hf * 128 + t) for key `key` of the unit
         auto grad_off = [&](int key, int hf) {
@@ -144,7 +153,8 @@ __device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base,
         if (u.T == 0) {  // keys that no query of the sequence sees: zero gradients
             T* dst = static_cast<T*>(half == 0 ? p.dv : p.dk);
             for (int key = u.n * 64; key < min(u.n * 64 + 64, u.Sk); ++key)
-                for (int hf = 0; hf < 2; ++hf) dst[grad_off(key, hf)] = static_cast<T>(0.0f);
+                for (int hf = 0; hf < 2; ++hf)
+                    if (D == 256 || hf * 128 + t < D) dst[grad_off(key, hf)] = static_cast<T>(0.0f);
             continue;
         }
         for (int s = 0; s < u.T; ++s, ++it) {
@@ -220,6 +230,8 @@ __device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base,
             T* dst = static_cast<T*>(which == 0 ? p.dv : p.dk);
 #pragma unroll 1
             for (int hf = 0; hf < 2; ++hf) {
+                if constexpr (D < 256)
+                    if (hf * 128 + t >= D) break;  // a zero lane of the padded half
                 const uint32_t col = (which == 0 ? C::T_DV : C::T_DK) + hf * 64;
                 uint32_t r[32];
 #pragma unroll 1
@@ -238,17 +250,17 @@ __device__ void bwd256_compute(const BwdParams& p, uint32_t tmem, uint32_t base,
 }
 
 // ---- dQ warpgroup: two 128-dim halves of dQ^T per step -> fp32 reductions -----------
-template <bool BF16>
-__device__ void bwd256_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int wq)
+template <int D, bool BF16>
+__device__ void bwd_wide_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int wq)
 {
-    using C = Bwd256Cfg<BF16>;
+    using C = BwdWideCfg<D, BF16>;
     const int lane = threadIdx.x & 31;
     const int t = wq * 32 + lane;  // head dim within the half (= TMEM lane of dQ^T)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     auto bar = [&](int i) { return bars + 8u * i; };
     uint32_t k = 0;  // dQ halves drained so far
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
-        const BwdUnit u = bwd256_decode(p, ui);
+        const BwdUnit u = bwd_wide_decode(p, ui);
         for (int s = 0; s < u.T; ++s) {
             int h, m;
             bwd_step(p, u, s, h, m);
@@ -256,6 +268,12 @@ __device__ void bwd256_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bar
 #pragma unroll 1
             for (int dh = 0; dh < 2; ++dh, ++k) {
                 if (!warp_wait<true>(bar(C::B_DQ_FULL), k & 1u, ctl, W_B256_DQ_FULL)) return;
+                if constexpr (D < 256) {
+                    if (dh * 128 + wq * 32 >= D) {  // zero lanes of the padded half
+                        if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
+                        continue;
+                    }
+                }
                 tc_fence_after();
                 uint32_t r[128];  // r[i] = dQ^T[dim dh*128 + t][query i]
                 tmem_ld128_split(tmem + lane_off + C::T_DQ, r);
@@ -270,10 +288,10 @@ __device__ void bwd256_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bar
 }
 
 // ---- MMA issuer ----------------------------------------------------------------------
-template <bool BF16>
-__device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars, CtaCtl* ctl)
+template <int D, bool BF16>
+__device__ void bwd_wide_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32_t bars, CtaCtl* ctl)
 {
-    using C = Bwd256Cfg<BF16>;
+    using C = BwdWideCfg<D, BF16>;
     using I = Issuer<C::WARP_ISSUE, true>;
     auto bar = [&](int i) { return bars + 8u * i; };
     const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQ = base + C::OFF_Q,
@@ -285,16 +303,16 @@ __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uin
     const uint64_t mQ = sdesc_sw128(sQ, C::Q_BLK, 1024), mDO = sdesc_sw128(sDO, C::Q_BLK, 1024);
     const uint64_t mP = sdesc_sw128(sP, C::Q_BLK, 1024), mDS = sdesc_sw128(sDS, C::Q_BLK, 1024);
     const uint64_t kDS = sdesc_sw128(sDS, 16, 1024), mK = sdesc_sw128(sK, C::KV_BLK, 1024);
-    // S (or dP) = X Y^T over d = 256: X a [128][256] tile, Y a [64][256] tile
+    // S (or dP) = X Y^T over d: X a [128][d] tile, Y a [64][d] tile
     auto mma_qk = [&](uint32_t d_t, uint64_t x, uint64_t y) {
 #pragma unroll
-        for (int kk = 0; kk < 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t xo = ((kk >> 2) * C::Q_BLK + (kk & 3) * 32u) >> 4;
             const uint32_t yo = ((kk >> 2) * C::KV_BLK + (kk & 3) * 32u) >> 4;
             I::ss(tmem + d_t, x + xo, y + yo, C::IDESC_S, kk > 0);
         }
     };
-    // acc^T[half] (+)= X^T Z: X a [128 query][256] tile read MN-major (head-dim half
+    // acc^T[half] (+)= X^T Z: X a [128 query][d] tile read MN-major (head-dim half
     // `hf`), Z a [128 query][64 key] tile read MN-major
     auto mma_t = [&](uint32_t d_t, uint64_t x, uint64_t z, bool acc) {
 #pragma unroll
@@ -317,7 +335,7 @@ __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uin
         return I::wait(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_B256_DQ_EMPTY);
     };
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
-        const BwdUnit u = bwd256_decode(p, ui);
+        const BwdUnit u = bwd_wide_decode(p, ui);
         if (u.T == 0) continue;
         if (!I::wait(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_B256_KV_FULL)) return;
         tc_fence_after();
@@ -368,9 +386,9 @@ __device__ void bwd256_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uin
 }
 
 // ---- TMA producer --------------------------------------------------------------------
-template <bool BF16>
-struct Bwd256Load {
-    using C = Bwd256Cfg<BF16>;
+template <int D, bool BF16>
+struct BwdWideLoad {
+    using C = BwdWideCfg<D, BF16>;
     const CUtensorMap *tmQ, *tmK, *tmV, *tmDO;  // K, V maps have 64-row boxes
     uint32_t base, bars;
     CtaCtl* ctl;
@@ -381,11 +399,11 @@ struct Bwd256Load {
     {
         uint32_t it = 0, unit_it = 0;
         for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
-            const BwdUnit u = bwd256_decode(p, ui);
+            const BwdUnit u = bwd_wide_decode(p, ui);
             if (u.T == 0) continue;
             if (!wait_bar_inl(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_B256_KV_EMPTY)) return;
-            mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::KV_BYTES);
-            for (int blk = 0; blk < 4; ++blk) {
+            mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::KV_LOAD);
+            for (int blk = 0; blk < C::NB; ++blk) {
                 tma_load_4d(base + C::OFF_K + blk * C::KV_BLK, tmK, bar(C::B_KV_FULL), blk * 64, u.hkv,
                             u.k_base + u.n * 64, u.tb);
                 tma_load_4d(base + C::OFF_V + blk * C::KV_BLK, tmV, bar(C::B_KV_FULL), blk * 64, u.hkv,
@@ -398,8 +416,8 @@ struct Bwd256Load {
                 bwd_step(p, u, s, h, m);
                 const uint32_t ph = (it & 1u) ^ 1u;
                 if (!wait_bar_inl(bar(C::B_Q_EMPTY), ph, ctl, W_B256_Q_EMPTY)) return;
-                mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_BYTES + C::ROWS_BYTES);
-                for (int blk = 0; blk < 4; ++blk)
+                mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_LOAD + C::ROWS_BYTES);
+                for (int blk = 0; blk < C::NB; ++blk)
                     tma_load_4d(base + C::OFF_Q + blk * C::Q_BLK, tmQ, bar(C::B_Q_FULL), blk * 64, h,
                                 u.q_base + m * 128, u.tb);
                 {
@@ -409,8 +427,8 @@ struct Bwd256Load {
                 }
                 q_round = static_cast<int>(it);
                 if (!wait_bar_inl(bar(C::B_DO_EMPTY), ph, ctl, W_B256_DO_EMPTY)) return;
-                mbar_arrive_expect_tx(bar(C::B_DO_FULL), C::Q_BYTES);
-                for (int blk = 0; blk < 4; ++blk)
+                mbar_arrive_expect_tx(bar(C::B_DO_FULL), C::Q_LOAD);
+                for (int blk = 0; blk < C::NB; ++blk)
                     tma_load_4d(base + C::OFF_DO + blk * C::Q_BLK, tmDO, bar(C::B_DO_FULL), blk * 64, h,
                                 u.q_base + m * 128, u.tb);
                 do_round = static_cast<int>(it);
@@ -425,13 +443,13 @@ struct Bwd256Load {
     }
 };
 
-template <bool BF16>
-__global__ void __launch_bounds__(Bwd256Cfg<BF16>::THREADS, 1)
-    fa_bwd_dkdv256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+template <int D, bool BF16>
+__global__ void __launch_bounds__(BwdWideCfg<D, BF16>::THREADS, 1)
+    fa_bwd_dkdv_wide_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                           const BwdParams p)
 {
-    using C = Bwd256Cfg<BF16>;
+    using C = BwdWideCfg<D, BF16>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
     if (base & 1023u) {  // swizzled TMA tiles and MMA descriptors need 1024-byte alignment
@@ -463,6 +481,19 @@ __global__ void __launch_bounds__(Bwd256Cfg<BF16>::THREADS, 1)
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmDO);
     }
+    if constexpr (C::NB < 4) {
+        // the fourth 64-dim block of K, V, Q and dO: zero, read by the tensor core only
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        for (uint32_t o = threadIdx.x * 16u; o < C::KV_BLK; o += C::THREADS * 16u) {
+            *reinterpret_cast<uint4*>(smem_raw + C::OFF_K + 3 * C::KV_BLK + o) = z;
+            *reinterpret_cast<uint4*>(smem_raw + C::OFF_V + 3 * C::KV_BLK + o) = z;
+        }
+        for (uint32_t o = threadIdx.x * 16u; o < C::Q_BLK; o += C::THREADS * 16u) {
+            *reinterpret_cast<uint4*>(smem_raw + C::OFF_Q + 3 * C::Q_BLK + o) = z;
+            *reinterpret_cast<uint4*>(smem_raw + C::OFF_DO + 3 * C::Q_BLK + o) = z;
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -471,22 +502,22 @@ __global__ void __launch_bounds__(Bwd256Cfg<BF16>::THREADS, 1)
     // register split (setmaxnreg, per warpgroup): warps 12-15 release registers on entry
     // to their branch, unconditionally, so the dQ warpgroup's increase always completes
     if (warp < C::DQ_WARP) {
-        bwd256_compute<BF16>(p, tmem, base, bars, ctl, warp & 3, warp >> 2);
+        bwd_wide_compute<D, BF16>(p, tmem, base, bars, ctl, warp & 3, warp >> 2);
     } else if (warp < C::MMA_WARP) {
         setmaxnreg_inc<C::REG_DQ>();  // completes once warps 12-15 have released theirs
-        bwd256_dq_reduce<BF16>(p, tmem, bars, ctl, warp - C::DQ_WARP);
+        bwd_wide_dq_reduce<D, BF16>(p, tmem, bars, ctl, warp - C::DQ_WARP);
     } else {
         setmaxnreg_dec<C::REG_CTRL>();  // all four warps, first thing, unconditionally
         if (warp == C::MMA_WARP) {
             if (C::WARP_ISSUE || lane == 0) {
-                bwd256_mma<BF16>(p, tmem, base, bars, ctl);
+                bwd_wide_mma<D, BF16>(p, tmem, base, bars, ctl);
                 Issuer<C::WARP_ISSUE, true>::commit(bars + 8u * C::B_DRAIN);
                 if (lane == 0) drain_wait_inl(bars + 8u * C::B_DRAIN, 0u, W_B256_DRAIN);
             }
             __syncwarp();
         } else if (warp == C::LOAD_WARP) {
             if (lane == 0) {
-                Bwd256Load<BF16> ld{&tmQ, &tmK, &tmV, &tmDO, base, bars, ctl};
+                BwdWideLoad<D, BF16> ld{&tmQ, &tmK, &tmV, &tmDO, base, bars, ctl};
                 ld.run(p);
                 ld.drain();
             }

@@ -82,11 +82,13 @@ enum : uint32_t {
 
 template <int D, bool BF16>
 struct FwdCfg {
-    static_assert(D == 128 || D == 256, "head_dim");
+    static_assert(D == 128 || D == 192 || D == 256, "head_dim");
     static constexpr int NQ = D == 128 ? 2 : 1;  // 128-row Q tiles per work unit
     static constexpr int NS = D == 128 ? 1 : 2;  // S buffers per Q tile
-    static constexpr int KCH = D / 128;          // 32-KB chunks per K (or V) tile
-    static constexpr int NSTAGE = 5;             // ring depth, in chunks
+    // ring chunk: 128 rows x CHUNK_COLS head dims (one or two 64-column swizzle atoms)
+    static constexpr int CHUNK_COLS = D == 192 ? 64 : 128;
+    static constexpr int KCH = D / CHUNK_COLS;    // chunks per K (or V) tile
+    static constexpr int NSTAGE = D == 192 ? 11 : 5;  // ring depth, in chunks
     static constexpr int BM = 128;               // query rows per Q tile
     static constexpr int BN = 128;               // keys per KV tile
     static constexpr int POLY_EVERY = 0;         // exp2 pairs: 1 in POLY_EVERY on the FMA pipe (0: none)
@@ -94,7 +96,7 @@ struct FwdCfg {
     // spinning waits (see fa_common.cuh) for the softmax and MMA warps
     static constexpr bool SPIN = D == 128;
     static constexpr int UNIT_ROWS = NQ * BM;
-    static constexpr uint32_t CHUNK = 32768;
+    static constexpr uint32_t CHUNK = BN * CHUNK_COLS * 2;
     static constexpr uint32_t QTILE = BM * D * 2;
     static constexpr uint32_t Q_BYTES = NQ * QTILE;
     static constexpr int SOFTMAX_WARPS = NQ * 4;     // one warpgroup per Q tile
@@ -129,7 +131,7 @@ struct FwdCfg {
     __device__ static constexpr uint32_t col_Pk(int kk) { return kk * 8; }
 
     static constexpr uint32_t IDESC_S = idesc_f16(BF16, 128, 128, false, false);
-    static constexpr uint32_t IDESC_PV = idesc_f16(BF16, 128, 128, false, true);
+    static constexpr uint32_t IDESC_PV = idesc_f16(BF16, 128, CHUNK_COLS, false, true);
 };
 
 template <int UNIT_ROWS>
@@ -399,7 +401,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
 }
 
 // ---------------------------------------------------------------------------------
-// MMA issuer.  head_dim 256: the whole warp runs the issue loop, converged, and each
+// MMA issuer.  head_dim 192 / 256: the whole warp runs the issue loop, converged, and each
 // tcgen05 op is executed by one elected lane (warp-uniform descriptors, few
 // instructions per MMA).  head_dim 128: lane 0 alone runs it (the converged form
 // measured about half as fast there).
@@ -407,7 +409,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
 template <int D, bool BF16>
 struct FwdMma {
     using C = FwdCfg<D, BF16>;
-    static constexpr bool WARP_ISSUE = D == 256;
+    static constexpr bool WARP_ISSUE = D != 128;
     using I = Issuer<WARP_ISSUE, false, C::SPIN>;
     uint32_t tmem, sQ, sRing, bars;
     CtaCtl* ctl;
@@ -449,15 +451,16 @@ struct FwdMma {
         uint64_t kd[C::KCH];
 #pragma unroll
         for (int c = 0; c < C::KCH; ++c) kd[c] = kdesc0 + slot_off(sK + c);
+        constexpr int KPC = C::CHUNK_COLS / 16;  // k-steps per chunk
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t aoff = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
-            const uint32_t boff = (((kk & 7) >> 2) * 16384u + (kk & 3) * 32u) >> 4;
-            ss(d, qd + aoff, kd[kk >> 3] + boff, C::IDESC_S, kk > 0);
+            const uint32_t boff = (((kk % KPC) >> 2) * 16384u + (kk & 3) * 32u) >> 4;
+            ss(d, qd + aoff, kd[kk / KPC] + boff, C::IDESC_S, kk > 0);
         }
     }
     // O_q (+)= P(q, sb) V, V tile in ring chunks sV .. sV + KCH - 1 (chunk c = O columns
-    // c*128 .. c*128+127)
+    // c*CHUNK_COLS .. (c+1)*CHUNK_COLS-1)
     __device__ void issue_PV(int q, int sb, uint32_t sV, bool acc)
     {
         uint64_t vd[C::KCH];
@@ -471,7 +474,7 @@ struct FwdMma {
             const uint32_t a = tP + C::col_Pk(kk);
 #pragma unroll
             for (int c = 0; c < C::KCH; ++c)
-                ts(tO + c * 128, a, vd[c] + (kk * 2048u >> 4), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                ts(tO + c * C::CHUNK_COLS, a, vd[c] + (kk * 2048u >> 4), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
     }
     __device__ bool wait_chunks(uint32_t s0)
@@ -614,15 +617,16 @@ struct FwdLoad {
         }
         const uint32_t dst = sRing + slot * C::CHUNK;
         mbar_arrive_expect_tx(bar(C::B_FULL + slot), C::CHUNK);
-        tma_load_4d(dst, tm, bar(C::B_FULL + slot), col0, hkv, row0, b);
-        tma_load_4d(dst + 16384u, tm, bar(C::B_FULL + slot), col0 + 64, hkv, row0, b);
+#pragma unroll
+        for (int a = 0; a < C::CHUNK_COLS / 64; ++a)
+            tma_load_4d(dst + a * 16384u, tm, bar(C::B_FULL + slot), col0 + 64 * a, hkv, row0, b);
         filled[slot] = static_cast<int>(round);
         return true;
     }
     __device__ bool load_kv(const CUtensorMap* tm, int row0, int hkv, int b)
     {
         for (int c = 0; c < C::KCH; ++c)
-            if (!load_chunk(tm, row0, c * 128, hkv, b)) return false;
+            if (!load_chunk(tm, row0, c * C::CHUNK_COLS, hkv, b)) return false;
         return true;
     }
 
@@ -787,12 +791,10 @@ __global__ void __launch_bounds__(256) fa_fwd_combine_kernel(const FwdParams p)
             sum += w;
             const float* src = p.opart + (static_cast<size_t>(s) * rows + row) * D + lane * PER;
 #pragma unroll
-            for (int c = 0; c < PER; c += 4) {
-                const float4 x = *reinterpret_cast<const float4*>(src + c);
+            for (int c = 0; c < PER; c += 2) {  // 8-byte loads: PER is 4, 6 or 8
+                const float2 x = *reinterpret_cast<const float2*>(src + c);
                 acc[c] = fmaf(w, x.x, acc[c]);
                 acc[c + 1] = fmaf(w, x.y, acc[c + 1]);
-                acc[c + 2] = fmaf(w, x.z, acc[c + 2]);
-                acc[c + 3] = fmaf(w, x.w, acc[c + 3]);
             }
         }
     }
@@ -803,8 +805,11 @@ __global__ void __launch_bounds__(256) fa_fwd_combine_kernel(const FwdParams p)
     for (int c = 0; c < PER / 2; ++c) w[c] = pack2<BF16>(acc[2 * c] * inv, acc[2 * c + 1] * inv);
     if constexpr (PER == 4) {
         *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
-    } else {
+    } else if constexpr (PER == 8) {
         *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {  // 12 bytes per lane: 4-byte aligned only
+#pragma unroll
+        for (int c = 0; c < PER / 2; ++c) reinterpret_cast<uint32_t*>(dst)[c] = w[c];
     }
     if (lane == 0)
         p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Sq + i] = m == -INFINITY ? -INFINITY : m + logf(sum);

@@ -23,9 +23,10 @@
  *     reads key/value head h / (Hq / Hkv).
  *   - causal != 0 applies a lower-triangular mask aligned to the bottom-right
  *     corner: key j is visible to query i iff j <= i + (Sk - Sq).
- *   - head_dim d must be 128 or 256; dtype must be FA_BF16 or FA_FP16 and is
- *     the same for every 16-bit tensor of a call.  Every pointer must be
- *     16-byte aligned.
+ *   - head_dim d must be 128, 192 or 256 (192: "[RFC] FA4 -- head_dim=256 &
+ *     head_dim=512", Phase 4, symmetric head_dim=192); dtype must be FA_BF16 or
+ *     FA_FP16 and is the same for every 16-bit tensor of a call.  Every pointer
+ *     must be 16-byte aligned.
  *   - Ownership: the caller owns every buffer.  The library allocates no device
  *     memory per call; scratch for the backward is the caller's workspace.
  *     Work is enqueued on `stream` and runs asynchronously; nothing synchronises.

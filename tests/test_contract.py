@@ -90,7 +90,7 @@ def bwd_call(lib, **kw):
     (dict(scale=float("nan")), FA_ERR_INVALID_ARG),
     (dict(scale=float("inf")), FA_ERR_INVALID_ARG),
     (dict(d=64), FA_ERR_UNSUPPORTED),
-    (dict(d=192), FA_ERR_UNSUPPORTED),
+    (dict(d=384), FA_ERR_UNSUPPORTED),
     (dict(d=512), FA_ERR_UNSUPPORTED),
     (dict(dt=2), FA_ERR_UNSUPPORTED),
     (dict(q=FAKE + 2), FA_ERR_INVALID_ARG),

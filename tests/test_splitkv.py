@@ -33,7 +33,7 @@ def test_splitkv_workspace_size(lib):
         rows = s * B * Hq * Sq
         assert lib.fa_fwd_splitkv_workspace_size(B, Sq, Sk, Hq, Hkv, d, s) == r256(rows * d * 4) + r256(rows * 4)
     assert lib.fa_fwd_splitkv_workspace_size(1, 1, 1, 3, 2, 128, 2) == 0   # Hq % Hkv
-    assert lib.fa_fwd_splitkv_workspace_size(1, 1, 1, 2, 2, 192, 2) == 0   # head dim
+    assert lib.fa_fwd_splitkv_workspace_size(1, 1, 1, 2, 2, 384, 2) == 0   # head dim
 
 
 def test_splitkv_rejections(lib):
