@@ -116,6 +116,17 @@ fa_status set_smem(K kernel, uint32_t bytes)
                : FA_ERR_CUDA;
 }
 
+// A kernel that moves registers between warpgroups with setmaxnreg assumes the launch
+// gives every thread exactly `launch_regs`; a build compiled to another count could
+// leave an increase waiting forever, so it is refused before any launch.
+template <typename K>
+fa_status check_regs(K kernel, int launch_regs)
+{
+    cudaFuncAttributes a{};
+    if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) return FA_ERR_CUDA;
+    return a.numRegs == launch_regs ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
 int g_inject = 0;
 std::mutex g_inject_mu;
 
@@ -133,11 +144,13 @@ fa_status launch_bwd_d128(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                           cudaStream_t stream)
 {
     using C = fa::BwdCfg<BF16>;
+    static const fa_status regs_ok = check_regs(fa::fa_bwd_dkdv_kernel<BF16>, C::REG_LAUNCH);
+    if (regs_ok != FA_OK) return regs_ok;
+    fa_status st = set_smem(fa::fa_bwd_dkdv_kernel<BF16>, C::SMEM_BYTES);
+    if (st != FA_OK) return st;
     const long long pre_rows = (long long)p.B * p.Hq * p.Sq_pad;
     fa::fa_bwd_pre_kernel<128, BF16><<<(unsigned)((pre_rows + 7) / 8), 256, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    fa_status st = set_smem(fa::fa_bwd_dkdv_kernel<BF16>, C::SMEM_BYTES);
-    if (st != FA_OK) return st;
     const int grid = p.num_units < sm_count ? p.num_units : sm_count;
     fa::fa_bwd_dkdv_kernel<BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -152,11 +165,13 @@ fa_status launch_bwd_wide(const CUtensorMap& tq, const CUtensorMap& tk64, const 
                           cudaStream_t stream)
 {
     using C = fa::BwdWideCfg<D, BF16>;
+    static const fa_status regs_ok = check_regs(fa::fa_bwd_dkdv_wide_kernel<D, BF16>, C::REG_LAUNCH);
+    if (regs_ok != FA_OK) return regs_ok;
+    fa_status st = set_smem(fa::fa_bwd_dkdv_wide_kernel<D, BF16>, C::SMEM_BYTES);
+    if (st != FA_OK) return st;
     const long long pre_rows = (long long)p.B * p.Hq * p.Sq_pad;
     fa::fa_bwd_pre_kernel<D, BF16><<<(unsigned)((pre_rows + 7) / 8), 256, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    fa_status st = set_smem(fa::fa_bwd_dkdv_wide_kernel<D, BF16>, C::SMEM_BYTES);
-    if (st != FA_OK) return st;
     const int grid = p.num_units < sm_count ? p.num_units : sm_count;
     fa::fa_bwd_dkdv_wide_kernel<D, BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk64, tv64, tdo, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -170,6 +185,10 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
                      fa::FwdParams p, int sm_count, cudaStream_t stream)
 {
     using C = fa::FwdCfg<D, BF16>;
+    if constexpr (C::REG_SPLIT) {
+        static const fa_status regs_ok = check_regs(fa::fa_fwd_kernel<D, BF16>, C::REG_LAUNCH);
+        if (regs_ok != FA_OK) return regs_ok;
+    }
     fa_status st = set_smem(fa::fa_fwd_kernel<D, BF16>, C::SMEM_BYTES);
     if (st != FA_OK) return st;
 

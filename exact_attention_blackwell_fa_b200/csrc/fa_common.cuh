@@ -84,6 +84,21 @@ __device__ __noinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32_t 
     return drain_wait_inl(bar, parity, where);
 }
 
+// The timed waits, inlined (INL) or called.  Code that runs under a setmaxnreg budget
+// other than the launch's must not call functions, so it takes the inlined form.
+template <bool INL>
+__device__ __forceinline__ bool wait_bar_t(uint32_t bar, uint32_t parity, CtaCtl* ctl, uint32_t where)
+{
+    if constexpr (INL) return wait_bar_inl(bar, parity, ctl, where);
+    else return wait_bar(bar, parity, ctl, where);
+}
+template <bool INL>
+__device__ __forceinline__ bool drain_wait_t(uint32_t bar, uint32_t parity, uint32_t where)
+{
+    if constexpr (INL) return drain_wait_inl(bar, parity, where);
+    else return drain_wait(bar, parity, where);
+}
+
 // Single-thread wait: one inline probe (SPIN: a bounded non-suspending poll), then the
 // timed wait.
 template <bool INL = false, bool SPIN = false>

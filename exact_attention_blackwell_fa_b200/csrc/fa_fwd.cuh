@@ -101,7 +101,17 @@ struct FwdCfg {
     static constexpr uint32_t Q_BYTES = NQ * QTILE;
     static constexpr int SOFTMAX_WARPS = NQ * 4;     // one warpgroup per Q tile
     static constexpr int CTRL_WARP = SOFTMAX_WARPS;  // MMA warp; the TMA warp follows it
-    static constexpr int THREADS = (SOFTMAX_WARPS + 2) * 32;
+    // head_dim 128: the MMA and TMA warps plus two idle ones form a whole warpgroup,
+    // which hands registers to the two softmax warpgroups (setmaxnreg); the launch
+    // budget is 65536 / 384 = 168 per thread, and the host refuses to launch a build
+    // whose register count differs (the increase would never be granted)
+    static constexpr bool REG_SPLIT = D == 128;
+    static constexpr int THREADS = (SOFTMAX_WARPS + (REG_SPLIT ? 4 : 2)) * 32;
+    static constexpr uint32_t REG_LAUNCH = 168, REG_SOFTMAX = 192, REG_CTRL = 120;
+    static_assert(!REG_SPLIT || (THREADS == 384 && SOFTMAX_WARPS * 32 * REG_SOFTMAX + 4 * 32 * REG_CTRL <=
+                                                       THREADS * REG_LAUNCH),
+                  "register split exceeds the launch budget");
+    static constexpr bool INL = REG_SPLIT;  // inlined waits (no calls under setmaxnreg)
 
     // shared memory map (offsets from the 1024-aligned dynamic shared memory base)
     static constexpr uint32_t OFF_Q = 0;
@@ -267,7 +277,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
         for (int j = 0; j < n; ++j, ++s_it) {
             const int sb = s_it % C::NS;
             const uint32_t tS = tmem + lane_off + C::col_S(q, sb);
-            if (!warp_wait<false, C::SPIN>(bar(C::B_S_FULL + q * C::NS + sb), (s_it / C::NS) & 1u, ctl, W_FWD_S_FULL))
+            if (!warp_wait<C::INL, C::SPIN>(bar(C::B_S_FULL + q * C::NS + sb), (s_it / C::NS) & 1u, ctl, W_FWD_S_FULL))
                 return;
             tc_fence_after();
             uint32_t sr[128];
@@ -337,7 +347,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
             // wait for the previous P V (the MMA commits O_done after each one)
             if (__any_sync(0xffffffffu, resc)) {
                 if (C::NS == 2) {
-                    if (!warp_wait<false, C::SPIN>(bar(C::B_O_DONE + q), (s_it - 1u) & 1u, ctl, W_FWD_O_DONE))
+                    if (!warp_wait<C::INL, C::SPIN>(bar(C::B_O_DONE + q), (s_it - 1u) & 1u, ctl, W_FWD_O_DONE))
                         return;
                     tc_fence_after();
                 }
@@ -357,7 +367,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
             if (lane == 0) mbar_arrive(bar(C::B_P_FULL + q * C::NS + sb));
         }
         // epilogue: wait for the unit's last P V, normalise and store O and LSE
-        if (!warp_wait<false, C::SPIN>(bar(C::B_O_FINAL + q), tile_it & 1u, ctl, W_FWD_O_FINAL)) return;
+        if (!warp_wait<C::INL, C::SPIN>(bar(C::B_O_FINAL + q), tile_it & 1u, ctl, W_FWD_O_FINAL)) return;
         ++tile_it;
         tc_fence_after();
         const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
@@ -410,7 +420,7 @@ template <int D, bool BF16>
 struct FwdMma {
     using C = FwdCfg<D, BF16>;
     static constexpr bool WARP_ISSUE = D != 128;
-    using I = Issuer<WARP_ISSUE, false, C::SPIN>;
+    using I = Issuer<WARP_ISSUE, C::INL, C::SPIN>;
     uint32_t tmem, sQ, sRing, bars;
     CtaCtl* ctl;
     uint32_t seq = 0;  // ring chunk sequence number
@@ -610,7 +620,7 @@ struct FwdLoad {
         const uint32_t s = seq++;
         const int slot = s % C::NSTAGE;
         const uint32_t round = s / C::NSTAGE;
-        if (!wait_bar(bar(C::B_EMPTY + slot), (round & 1u) ^ 1u, ctl, W_FWD_RING_EMPTY)) return false;
+        if (!wait_bar_t<C::INL>(bar(C::B_EMPTY + slot), (round & 1u) ^ 1u, ctl, W_FWD_RING_EMPTY)) return false;
         if (inject) {  // test hook: never fill this chunk; its consumer times out
             inject = 0;
             return true;
@@ -643,7 +653,7 @@ struct FwdLoad {
             // rows past the sequence's end (the next sequence's, or out of range) are
             // loaded too: their scores are masked, their outputs never stored
             auto krow = [&](int j) { return u.k_base + (u.j0 + j) * C::BN; };
-            if (!wait_bar(bar(C::B_Q_EMPTY), (q_it & 1u) ^ 1u, ctl, W_FWD_Q_EMPTY)) return;
+            if (!wait_bar_t<C::INL>(bar(C::B_Q_EMPTY), (q_it & 1u) ^ 1u, ctl, W_FWD_Q_EMPTY)) return;
             mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_BYTES);
             // packing: one box spans the group's `pack` heads x BM / pack queries, so
             // shared-memory row r holds query r / pack of head r % pack
@@ -675,8 +685,9 @@ struct FwdLoad {
     __device__ void drain()
     {
         for (int i = 0; i < C::NSTAGE; ++i)
-            if (filled[i] >= 0) drain_wait(bar(C::B_FULL + i), static_cast<uint32_t>(filled[i]) & 1u, W_FWD_DRAIN);
-        if (q_round >= 0) drain_wait(bar(C::B_Q_FULL), static_cast<uint32_t>(q_round) & 1u, W_FWD_DRAIN);
+            if (filled[i] >= 0)
+                drain_wait_t<C::INL>(bar(C::B_FULL + i), static_cast<uint32_t>(filled[i]) & 1u, W_FWD_DRAIN);
+        if (q_round >= 0) drain_wait_t<C::INL>(bar(C::B_Q_FULL), static_cast<uint32_t>(q_round) & 1u, W_FWD_DRAIN);
     }
 };
 
@@ -736,25 +747,29 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
     const uint32_t tmem = ctl->tmem_base;
 
     if (warp < C::SOFTMAX_WARPS) {
+        if constexpr (C::REG_SPLIT) setmaxnreg_inc<C::REG_SOFTMAX>();  // granted once warps 8-11 released theirs
         fwd_softmax_row<D, BF16>(p, tmem, bars, ctl, warp / 4, warp & 3);
-    } else if (warp == C::CTRL_WARP) {
-        using M = FwdMma<D, BF16>;
-        if (M::WARP_ISSUE || lane == 0) {
-            M mma{tmem, sQ, sRing, bars, ctl};
-            mma.init_descs();
-            mma.run(p);
-            // all MMAs issued by this warp must finish before TMEM is released
-            M::commit(bars + 8u * C::B_DRAIN);
-            if (lane == 0) drain_wait(bars + 8u * C::B_DRAIN, 0u, W_FWD_DRAIN);
+    } else {
+        if constexpr (C::REG_SPLIT) setmaxnreg_dec<C::REG_CTRL>();  // every control warp, first thing
+        if (warp == C::CTRL_WARP) {
+            using M = FwdMma<D, BF16>;
+            if (M::WARP_ISSUE || lane == 0) {
+                M mma{tmem, sQ, sRing, bars, ctl};
+                mma.init_descs();
+                mma.run(p);
+                // all MMAs issued by this warp must finish before TMEM is released
+                M::commit(bars + 8u * C::B_DRAIN);
+                if (lane == 0) drain_wait_t<C::INL>(bars + 8u * C::B_DRAIN, 0u, W_FWD_DRAIN);
+            }
+            __syncwarp();
+        } else if (warp == C::CTRL_WARP + 1) {
+            if (lane == 0) {
+                FwdLoad<D, BF16> ld{&tmQ, &tmK, &tmV, sQ, sRing, bars, ctl};
+                ld.run(p);
+                ld.drain();
+            }
+            __syncwarp();
         }
-        __syncwarp();
-    } else if (warp == C::CTRL_WARP + 1) {
-        if (lane == 0) {
-            FwdLoad<D, BF16> ld{&tmQ, &tmK, &tmV, sQ, sRing, bars, ctl};
-            ld.run(p);
-            ld.drain();
-        }
-        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
