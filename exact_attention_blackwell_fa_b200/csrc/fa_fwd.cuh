@@ -85,7 +85,10 @@ struct FwdCfg {
     static_assert(D == 128 || D == 192 || D == 256, "head_dim");
     static constexpr int NQ = D == 128 ? 2 : 1;  // 128-row Q tiles per work unit
     static constexpr int NS = D == 128 ? 1 : 2;  // S buffers per Q tile
-    // ring chunk: 128 rows x CHUNK_COLS head dims (one or two 64-column swizzle atoms)
+    // ring chunk: 128 rows x CHUNK_COLS head dims (one or two 64-column swizzle atoms).
+    // With one Q tile (d = 192, 256) each chunk is waited for just before and released
+    // just after the MMAs that read it, so the ring refills while the rest of the tile
+    // is still being read
     static constexpr int CHUNK_COLS = D == 192 ? 64 : 128;
     static constexpr int KCH = D / CHUNK_COLS;    // chunks per K (or V) tile
     static constexpr int NSTAGE = D == 192 ? 11 : 5;  // ring depth, in chunks
@@ -453,8 +456,10 @@ struct FwdMma {
         return static_cast<uint64_t>((s % C::NSTAGE) * (C::CHUNK >> 4));
     }
 
-    // S(q, sb) = Q_q K^T, K tile in ring chunks sK .. sK + KCH - 1
-    __device__ void issue_S(int q, int sb, uint32_t sK)
+    // S(q, sb) = Q_q K^T, K tile in ring chunks sK .. sK + KCH - 1.  STREAM: wait for
+    // each chunk right before its k-steps and release it right after them.
+    template <bool STREAM>
+    __device__ bool issue_S(int q, int sb, uint32_t sK)
     {
         const uint32_t d = tmem + C::col_S(q, sb);
         const uint64_t qd = qdesc0 + static_cast<uint64_t>(q * (C::QTILE >> 4));
@@ -464,28 +469,53 @@ struct FwdMma {
         constexpr int KPC = C::CHUNK_COLS / 16;  // k-steps per chunk
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
+            if constexpr (STREAM) {
+                if (kk % KPC == 0) {
+                    if (!wait_full(sK + kk / KPC)) return false;
+                    tc_fence_after();
+                }
+            }
             const uint32_t aoff = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
             const uint32_t boff = (((kk % KPC) >> 2) * 16384u + (kk & 3) * 32u) >> 4;
             ss(d, qd + aoff, kd[kk / KPC] + boff, C::IDESC_S, kk > 0);
+            if constexpr (STREAM)
+                if (kk % KPC == KPC - 1) release(sK + kk / KPC);
         }
+        return true;
     }
     // O_q (+)= P(q, sb) V, V tile in ring chunks sV .. sV + KCH - 1 (chunk c = O columns
     // c*CHUNK_COLS .. (c+1)*CHUNK_COLS-1)
-    __device__ void issue_PV(int q, int sb, uint32_t sV, bool acc)
+    // (k-steps 0-3 read P of key columns 0-63, 4-7 of 64-127.)  STREAM: chunk by chunk,
+    // each waited for before and released after its eight k-steps.
+    template <bool STREAM>
+    __device__ bool issue_PV(int q, int sb, uint32_t sV, bool acc)
     {
         uint64_t vd[C::KCH];
 #pragma unroll
         for (int c = 0; c < C::KCH; ++c) vd[c] = vdesc0 + slot_off(sV + c);
         const uint32_t tP = tmem + C::col_S(q, sb);
         const uint32_t tO = tmem + C::col_O(q);
+        if constexpr (STREAM) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            // k-steps 0-3 read P of key columns 0-63 (half 0), 4-7 of 64-127 (half 1)
-            const uint32_t a = tP + C::col_Pk(kk);
+            for (int c = 0; c < C::KCH; ++c) {
+                if (!wait_full(sV + c)) return false;
+                tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < C::KCH; ++c)
-                ts(tO + c * C::CHUNK_COLS, a, vd[c] + (kk * 2048u >> 4), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 8; ++kk)
+                    ts(tO + c * C::CHUNK_COLS, tP + C::col_Pk(kk), vd[c] + (kk * 2048u >> 4), C::IDESC_PV,
+                       (acc || kk > 0) ? 1u : 0u);
+                release(sV + c);
+            }
+        } else {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t a = tP + C::col_Pk(kk);
+#pragma unroll
+                for (int c = 0; c < C::KCH; ++c)
+                    ts(tO + c * C::CHUNK_COLS, a, vd[c] + (kk * 2048u >> 4), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+            }
         }
+        return true;
     }
     __device__ bool wait_chunks(uint32_t s0)
     {
@@ -515,7 +545,7 @@ struct FwdMma {
                 seq += 1;
                 if (!wait_chunks(sK)) return;
                 for (int q = 0; q < 2; ++q) {
-                    issue_S(q, 0, sK);
+                    issue_S<false>(q, 0, sK);
                     commit(bar(C::B_S_FULL + q));
                     ++s_it[q];
                 }
@@ -527,20 +557,20 @@ struct FwdMma {
                     if (!wait_chunks(sV)) return;
                     if (!wait(bar(C::B_P_FULL + 0), p_it[0] & 1u, W_FWD_P_FULL)) return;
                     tc_fence_after();
-                    issue_PV(0, 0, sV, j > 1);
+                    issue_PV<false>(0, 0, sV, j > 1);
                     ++p_it[0];
                     sK = seq;
                     seq += 1;
                     if (!wait_chunks(sK)) return;
-                    issue_S(0, 0, sK);
+                    issue_S<false>(0, 0, sK);
                     commit(bar(C::B_S_FULL + 0));
                     ++s_it[0];
                     if (!wait(bar(C::B_P_FULL + 1), p_it[1] & 1u, W_FWD_P_FULL)) return;
                     tc_fence_after();
-                    issue_PV(1, 0, sV, j > 1);
+                    issue_PV<false>(1, 0, sV, j > 1);
                     ++p_it[1];
                     release(sV);
-                    issue_S(1, 0, sK);
+                    issue_S<false>(1, 0, sK);
                     commit(bar(C::B_S_FULL + 1));
                     ++s_it[1];
                     release(sK);
@@ -552,7 +582,7 @@ struct FwdMma {
                 for (int q = 0; q < 2; ++q) {
                     if (!wait(bar(C::B_P_FULL + q), p_it[q] & 1u, W_FWD_P_FULL)) return;
                     tc_fence_after();
-                    issue_PV(q, 0, sV, n > 1);
+                    issue_PV<false>(q, 0, sV, n > 1);
                     ++p_it[q];
                     commit(bar(C::B_O_FINAL + q));
                 }
@@ -562,34 +592,28 @@ struct FwdMma {
                 for (int j = 0; j < 2 && j < n; ++j) {
                     const uint32_t sK = seq;
                     seq += C::KCH;
-                    if (!wait_chunks(sK)) return;
                     const int sb = s_it[0] & 1;
-                    issue_S(0, sb, sK);
+                    if (!issue_S<true>(0, sb, sK)) return;
                     commit(bar(C::B_S_FULL + sb));
                     ++s_it[0];
-                    release_chunks(sK);
                 }
                 if (n <= 2) commit(bar(C::B_Q_EMPTY));
                 for (int j = 0; j < n; ++j) {
                     const uint32_t sV = seq;
                     seq += C::KCH;
-                    if (!wait_chunks(sV)) return;
                     const int sbp = p_it[0] & 1;
                     if (!wait(bar(C::B_P_FULL + sbp), (p_it[0] >> 1) & 1u, W_FWD_P_FULL)) return;
                     tc_fence_after();
-                    issue_PV(0, sbp, sV, j > 0);
+                    if (!issue_PV<true>(0, sbp, sV, j > 0)) return;
                     commit(bar(C::B_O_DONE));
                     ++p_it[0];
-                    release_chunks(sV);
                     if (j + 2 < n) {
                         const uint32_t sK = seq;
                         seq += C::KCH;
-                        if (!wait_chunks(sK)) return;
                         const int sb = s_it[0] & 1;
-                        issue_S(0, sb, sK);
+                        if (!issue_S<true>(0, sb, sK)) return;
                         commit(bar(C::B_S_FULL + sb));
                         ++s_it[0];
-                        release_chunks(sK);
                         if (j + 2 == n - 1) commit(bar(C::B_Q_EMPTY));
                     }
                 }
