@@ -188,6 +188,8 @@ def main():
                          "decode-shaped")
     ap.add_argument("--splitkv", action="store_true",
                     help="forward through fa_fwd_splitkv (slice count chosen by the library)")
+    ap.add_argument("--clc", action="store_true",
+                    help="forward units ordered by cluster launch control (fa_set_unit_schedule)")
     ap.add_argument("--varlen", default=None,
                     help="comma-separated sequence lengths: one packed batch of these sequences "
                          "(fa_fwd_varlen / fa_bwd_varlen) instead of the dense workload")
@@ -233,6 +235,8 @@ def main():
                      "MiB each (L2: 126 MB)")}
     if lens:
         config["seq_lens"] = lens
+    if args.clc:
+        config["schedule"] = "cluster launch control"
 
     if args.impl == "reference":
         if rank != 0:
@@ -259,6 +263,9 @@ def main():
 
     import exact_attention_blackwell_fa_b200 as fa
     from exact_attention_blackwell_fa_b200.inputs import Shape, make_inputs
+
+    if args.clc:
+        fa.fa_set_unit_schedule(fa.FA_SCHED_CLC)
 
     if world > 1:
         import torch.distributed as dist

@@ -16,6 +16,7 @@ library's CUDA kernels.  The functions carry the C names:
     fa_status_string(code) -> str
     fa_last_device_status() -> (code, detail)
     fa_clear_device_status()
+    fa_set_unit_schedule(mode)        # FA_SCHED_STATIC (0, default) or FA_SCHED_CLC (1)
     fa_debug_inject(mode)
     fa_debug_exp2(x, mode=0) -> y
 
@@ -33,8 +34,11 @@ from . import _lib
 
 __all__ = [
     "FAError", "fa_fwd", "fa_fwd_splitkv", "fa_fwd_varlen", "fa_bwd", "fa_bwd_varlen", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
-    "fa_last_device_status", "fa_clear_device_status", "fa_debug_inject", "fa_debug_exp2",
+    "fa_last_device_status", "fa_clear_device_status", "fa_set_unit_schedule", "fa_debug_inject", "fa_debug_exp2",
+    "FA_SCHED_STATIC", "FA_SCHED_CLC",
 ]
+
+FA_SCHED_STATIC, FA_SCHED_CLC = 0, 1
 
 
 class FAError(RuntimeError):
@@ -260,6 +264,13 @@ def fa_last_device_status(stream=None):
 
 def fa_clear_device_status(stream=None):
     _raise(_lib.load().fa_clear_device_status(_stream_ptr(stream)), "fa_clear_device_status")
+
+
+def fa_set_unit_schedule(mode: int):
+    """Forward unit order: FA_SCHED_STATIC (persistent grid, fixed stride; default) or
+    FA_SCHED_CLC (one CTA per unit, running CTAs cancel pending ones to take their
+    units).  Process-wide."""
+    _raise(_lib.load().fa_set_unit_schedule(int(mode)), "fa_set_unit_schedule")
 
 
 def fa_debug_inject(mode: int):

@@ -36,6 +36,7 @@ SIGNATURES = {
     "fa_last_device_status": (_ci, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "fa_clear_device_status": (_ci, [_vp]),
     "fa_debug_inject": (_ci, [_ci]),
+    "fa_set_unit_schedule": (_ci, [_ci]),
     "fa_debug_exp2": (_ci, [_vp, _vp, _ci, _ci, _vp]),
 }
 

@@ -1,6 +1,7 @@
 // fa_api.cu -- the C ABI declared in include/fa.h: argument validation, TMA tensor
 // maps, device checks and kernel launches.  Every entry point validates first and
 // launches nothing on an invalid argument; there is no alternative code path.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -129,6 +130,7 @@ fa_status check_regs(K kernel, int launch_regs)
 
 int g_inject = 0;
 std::mutex g_inject_mu;
+std::atomic<int> g_schedule{FA_SCHED_STATIC};
 
 int take_inject()
 {
@@ -192,7 +194,8 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
     fa_status st = set_smem(fa::fa_fwd_kernel<D, BF16>, C::SMEM_BYTES);
     if (st != FA_OK) return st;
 
-    const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
+    // cluster launch control: one CTA per unit, the running ones take the rest
+    const int grid = p.clc ? p.num_tiles : (p.num_tiles < sm_count ? p.num_tiles : sm_count);
     fa::fa_fwd_kernel<D, BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -201,8 +204,11 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 int fwd_unit_rows(int d) { return d == 128 ? 256 : 128; }
 
 fa_status launch_fwd_any(int d, bool bf16, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const fa::FwdParams& p, int sm_count, cudaStream_t s)
+                         fa::FwdParams p, int sm_count, cudaStream_t s)
 {
+    // dynamic unit order (cluster launch control) when selected and there are more
+    // units than SMs
+    p.clc = (g_schedule.load(std::memory_order_relaxed) == FA_SCHED_CLC && p.num_tiles > sm_count) ? 1 : 0;
     switch (d) {
     case 128: return bf16 ? launch_fwd<128, true>(tq, tk, tv, p, sm_count, s) : launch_fwd<128, false>(tq, tk, tv, p, sm_count, s);
     case 192: return bf16 ? launch_fwd<192, true>(tq, tk, tv, p, sm_count, s) : launch_fwd<192, false>(tq, tk, tv, p, sm_count, s);
@@ -555,6 +561,13 @@ fa_status fa_debug_exp2(const float* x, float* y, int n, int mode, fa_stream str
     const int blocks = (pairs + threads - 1) / threads;
     fa::fa_debug_exp2_kernel<<<blocks, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n, mode);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_set_unit_schedule(int mode)
+{
+    if (mode != FA_SCHED_STATIC && mode != FA_SCHED_CLC) return FA_ERR_INVALID_ARG;
+    g_schedule.store(mode, std::memory_order_relaxed);
+    return FA_OK;
 }
 
 fa_status fa_debug_inject(int mode)

@@ -71,13 +71,17 @@ struct FwdParams {
     int causal;
     int inject;       // test hook: withhold the first K copy
     float sl2;        // scale * log2(e)
+    // clc != 0: the grid has one CTA per unit; a running CTA takes further units by
+    // cancelling CTAs that have not started (cluster launch control), in unit order.
+    // clc == 0: a persistent grid walks the units with a static stride.
+    int clc;
 };
 
 // wait-site codes reported through the device status word
 enum : uint32_t {
     W_FWD_Q_FULL = 0x101, W_FWD_Q_EMPTY, W_FWD_RING_FULL, W_FWD_RING_EMPTY, W_FWD_S_FULL,
     W_FWD_P_FULL, W_FWD_O_DONE, W_FWD_O_FINAL, W_FWD_DRAIN, W_FWD_RESERVED_A, W_FWD_RESERVED_B,
-    W_FWD_SMEM_ALIGN
+    W_FWD_SMEM_ALIGN, W_FWD_SCHED_FULL, W_FWD_SCHED_EMPTY, W_FWD_CLC
 };
 
 template <int D, bool BF16>
@@ -130,10 +134,20 @@ struct FwdCfg {
     static constexpr int B_O_DONE = B_P_FULL + NQ * NS;
     static constexpr int B_O_FINAL = B_O_DONE + NQ;
     static constexpr int B_DRAIN = B_O_FINAL + NQ;
-    static constexpr int NBAR = B_DRAIN + 1;
+    // unit schedule (clc): a ring of unit indices from the TMA thread to the softmax
+    // warps and the MMA warp, and the barrier of the cancellation response
+    static constexpr int NSCHED = 4;
+    static constexpr int B_SCHED_FULL = B_DRAIN + 1;
+    static constexpr int B_SCHED_EMPTY = B_SCHED_FULL + NSCHED;
+    static constexpr int B_CLC = B_SCHED_EMPTY + NSCHED;
+    static constexpr int NBAR = B_CLC + 1;
+    static constexpr int SCHED_READERS = SOFTMAX_WARPS + 1;  // arrivals that free a slot
     static constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
+    static constexpr uint32_t OFF_SCHED = (OFF_CTL + sizeof(CtaCtl) + 15u) & ~15u;  // int[NSCHED]
+    static constexpr uint32_t OFF_CLC = OFF_SCHED + 4 * NSCHED;                      // 16-byte response
     // no alignment slack: the kernel checks that the base is 1024-byte aligned
-    static constexpr uint32_t SMEM_BYTES = OFF_CTL + sizeof(CtaCtl);
+    static constexpr uint32_t SMEM_BYTES = OFF_CLC + 16;
+    static_assert(NSCHED * 4 % 16 == 0, "response alignment");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
     // TMEM columns
@@ -222,11 +236,64 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int t)
 }
 
 // ---------------------------------------------------------------------------------
+// The unit sequence one role walks.  Static: blockIdx.x, then every gridDim.x-th
+// unit.  Cluster launch control: the indices the TMA thread publishes in the
+// schedule ring, -1 ending it (-2: a wait gave up).  WARP: called by a whole
+// converged warp (lane 0 waits and frees the slot), else by one thread.
+// ---------------------------------------------------------------------------------
+template <int D, bool BF16, bool WARP>
+struct FwdUnits {
+    using C = FwdCfg<D, BF16>;
+    uint32_t bars, sched;
+    CtaCtl* ctl;
+    int clc;
+    int t = -1;
+    uint32_t k = 0;  // slots read
+
+    __device__ int first(const FwdParams& p)
+    {
+        if (!clc) {
+            t = blockIdx.x;
+            return t < p.num_tiles ? t : -1;
+        }
+        return read();
+    }
+    __device__ int next(const FwdParams& p)
+    {
+        if (!clc) {
+            t += gridDim.x;
+            return t < p.num_tiles ? t : -1;
+        }
+        return read();
+    }
+    __device__ int read()
+    {
+        const uint32_t slot = k % C::NSCHED, ph = (k / C::NSCHED) & 1u;
+        ++k;
+        const uint32_t full = bars + 8u * (C::B_SCHED_FULL + slot);
+        bool ok;
+        if constexpr (WARP) ok = warp_wait<C::INL, false>(full, ph, ctl, W_FWD_SCHED_FULL);
+        else ok = wait_bar_t<C::INL>(full, ph, ctl, W_FWD_SCHED_FULL);
+        if (!ok) return -2;
+        int v;
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(sched + 4u * slot) : "memory");
+        if constexpr (WARP) {
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(bars + 8u * (C::B_SCHED_EMPTY + slot));
+        } else {
+            mbar_arrive(bars + 8u * (C::B_SCHED_EMPTY + slot));
+        }
+        return v;
+    }
+};
+
+// ---------------------------------------------------------------------------------
 // Softmax / epilogue warpgroup, one per 128-row Q tile: thread = one query row, all
 // 128 key columns of a tile held in registers.
 // ---------------------------------------------------------------------------------
 template <int D, bool BF16>
-__device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars, CtaCtl* ctl, int q, int wq)
+__device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars, uint32_t sched, CtaCtl* ctl, int q,
+                                int wq)
 {
     using C = FwdCfg<D, BF16>;
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
@@ -238,7 +305,8 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
     const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
     uint32_t s_it = 0, tile_it = 0;
 
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+    FwdUnits<D, BF16, true> units{bars, sched, ctl, p.clc};
+    for (int t = units.first(p); t >= 0; t = units.next(p)) {
         const FwdUnit u = fwd_unit<C::UNIT_ROWS>(p, t);
         if (!u.rows) continue;  // past the end of its (shorter) sequence: nothing to do
         const int n = u.n;
@@ -424,7 +492,7 @@ struct FwdMma {
     using C = FwdCfg<D, BF16>;
     static constexpr bool WARP_ISSUE = D != 128;
     using I = Issuer<WARP_ISSUE, C::INL, C::SPIN>;
-    uint32_t tmem, sQ, sRing, bars;
+    uint32_t tmem, sQ, sRing, bars, sched;
     CtaCtl* ctl;
     uint32_t seq = 0;  // ring chunk sequence number
 
@@ -533,7 +601,8 @@ struct FwdMma {
     {
         uint32_t s_it[C::NQ] = {}, p_it[C::NQ] = {};
         uint32_t q_it = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+        FwdUnits<D, BF16, WARP_ISSUE> units{bars, sched, ctl, p.clc};
+        for (int t = units.first(p); t >= 0; t = units.next(p)) {
             const int n = fwd_unit<C::UNIT_ROWS>(p, t).n;
             if (n == 0) continue;
             if (!wait(bar(C::B_Q_FULL), q_it & 1u, W_FWD_Q_FULL)) return;
@@ -630,12 +699,15 @@ template <int D, bool BF16>
 struct FwdLoad {
     using C = FwdCfg<D, BF16>;
     const CUtensorMap *tmQ, *tmK, *tmV;
-    uint32_t sQ, sRing, bars;
+    uint32_t sQ, sRing, bars, sched;
     CtaCtl* ctl;
     uint32_t seq = 0;
     int filled[C::NSTAGE];  // ring round of the last fill per slot, -1 if none
     int q_round = -1;
     int inject = 0;
+    uint32_t pushed = 0;    // schedule slots written
+    uint32_t clc_it = 0;    // cancellation requests answered
+    bool clc_pending = false;
 
     __device__ uint32_t bar(int i) const { return bars + 8u * i; }
 
@@ -664,20 +736,60 @@ struct FwdLoad {
         return true;
     }
 
+    // publish the next unit index (or -1) to the softmax and MMA warps
+    __device__ bool push(int v)
+    {
+        const uint32_t slot = pushed % C::NSCHED, ph = ((pushed / C::NSCHED) & 1u) ^ 1u;
+        ++pushed;
+        if (!wait_bar_t<C::INL>(bar(C::B_SCHED_EMPTY + slot), ph, ctl, W_FWD_SCHED_EMPTY)) return false;
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sched + 4u * slot), "r"(v) : "memory");
+        mbar_arrive(bar(C::B_SCHED_FULL + slot));
+        return true;
+    }
+
     __device__ void run(const FwdParams& p)
     {
         for (int i = 0; i < C::NSTAGE; ++i) filled[i] = -1;
         inject = p.inject;
         uint32_t q_it = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+        const uint32_t resp = sched + 4u * C::NSCHED;  // the 16-byte cancellation response
+        int t = blockIdx.x;
+        if (t >= p.num_tiles) return;
+        if (p.clc && !push(t)) return;
+        while (true) {
+            if (p.clc) {  // ask for the next unit now; the answer is read after this one's loads
+                mbar_arrive_expect_tx(bar(C::B_CLC), 16);
+                clc_try_cancel(resp, bar(C::B_CLC));
+                clc_pending = true;
+            }
+            if (!load_unit(p, t, q_it)) return;
+            if (p.clc) {
+                if (!wait_bar_t<C::INL>(bar(C::B_CLC), clc_it & 1u, ctl, W_FWD_CLC)) return;
+                clc_pending = false;
+                ++clc_it;
+                int x;
+                t = clc_query(resp, x) ? x : -1;  // after a refusal, never ask again
+                if (!push(t)) return;
+                if (t < 0) return;
+            } else {
+                t += gridDim.x;
+                if (t >= p.num_tiles) return;
+            }
+        }
+    }
+
+    // Q and the K / V tiles of unit t, in the MMA issuer's order; false if a wait gave up
+    __device__ bool load_unit(const FwdParams& p, int t, uint32_t& q_it)
+    {
+        {
             const FwdUnit u = fwd_unit<C::UNIT_ROWS>(p, t);
             const int n = u.n, b = u.tb;
-            if (n == 0) continue;
+            if (n == 0) return true;
             const int hkv = p.pack > 1 ? u.h : u.h / p.group;
             // rows past the sequence's end (the next sequence's, or out of range) are
             // loaded too: their scores are masked, their outputs never stored
             auto krow = [&](int j) { return u.k_base + (u.j0 + j) * C::BN; };
-            if (!wait_bar_t<C::INL>(bar(C::B_Q_EMPTY), (q_it & 1u) ^ 1u, ctl, W_FWD_Q_EMPTY)) return;
+            if (!wait_bar_t<C::INL>(bar(C::B_Q_EMPTY), (q_it & 1u) ^ 1u, ctl, W_FWD_Q_EMPTY)) return false;
             mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_BYTES);
             // packing: one box spans the group's `pack` heads x BM / pack queries, so
             // shared-memory row r holds query r / pack of head r % pack
@@ -690,18 +802,19 @@ struct FwdLoad {
             ++q_it;
             if constexpr (C::NQ == 2) {
                 for (int j = 0; j < n; ++j) {
-                    if (!load_kv(tmK, krow(j), hkv, b)) return;
-                    if (!load_kv(tmV, krow(j), hkv, b)) return;
+                    if (!load_kv(tmK, krow(j), hkv, b)) return false;
+                    if (!load_kv(tmV, krow(j), hkv, b)) return false;
                 }
             } else {
                 for (int j = 0; j < 2 && j < n; ++j)
-                    if (!load_kv(tmK, krow(j), hkv, b)) return;
+                    if (!load_kv(tmK, krow(j), hkv, b)) return false;
                 for (int j = 0; j < n; ++j) {
-                    if (!load_kv(tmV, krow(j), hkv, b)) return;
-                    if (j + 2 < n && !load_kv(tmK, krow(j + 2), hkv, b)) return;
+                    if (!load_kv(tmV, krow(j), hkv, b)) return false;
+                    if (j + 2 < n && !load_kv(tmK, krow(j + 2), hkv, b)) return false;
                 }
             }
         }
+        return true;
     }
 
     // Before the CTA exits, wait for every copy this thread started (normally all
@@ -712,6 +825,8 @@ struct FwdLoad {
             if (filled[i] >= 0)
                 drain_wait_t<C::INL>(bar(C::B_FULL + i), static_cast<uint32_t>(filled[i]) & 1u, W_FWD_DRAIN);
         if (q_round >= 0) drain_wait_t<C::INL>(bar(C::B_Q_FULL), static_cast<uint32_t>(q_round) & 1u, W_FWD_DRAIN);
+        // an unanswered cancellation request still writes its response
+        if (clc_pending) drain_wait_t<C::INL>(bar(C::B_CLC), clc_it & 1u, W_FWD_DRAIN);
     }
 };
 
@@ -732,6 +847,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
     const uint32_t sQ = base + C::OFF_Q;
     const uint32_t sRing = base + C::OFF_RING;
     const uint32_t bars = base + C::OFF_BAR;
+    const uint32_t sched = base + C::OFF_SCHED;
     CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem_raw + C::OFF_CTL);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -753,6 +869,11 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
             mbar_init(bar(C::B_O_FINAL + q), 1);
         }
         mbar_init(bar(C::B_DRAIN), 1);
+        for (int i = 0; i < C::NSCHED; ++i) {
+            mbar_init(bar(C::B_SCHED_FULL + i), 1);
+            mbar_init(bar(C::B_SCHED_EMPTY + i), C::SCHED_READERS);
+        }
+        mbar_init(bar(C::B_CLC), 1);
         ctl->abort = 0u;
         fence_mbar_init();
     }
@@ -772,13 +893,13 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
 
     if (warp < C::SOFTMAX_WARPS) {
         if constexpr (C::REG_SPLIT) setmaxnreg_inc<C::REG_SOFTMAX>();  // granted once warps 8-11 released theirs
-        fwd_softmax_row<D, BF16>(p, tmem, bars, ctl, warp / 4, warp & 3);
+        fwd_softmax_row<D, BF16>(p, tmem, bars, sched, ctl, warp / 4, warp & 3);
     } else {
         if constexpr (C::REG_SPLIT) setmaxnreg_dec<C::REG_CTRL>();  // every control warp, first thing
         if (warp == C::CTRL_WARP) {
             using M = FwdMma<D, BF16>;
             if (M::WARP_ISSUE || lane == 0) {
-                M mma{tmem, sQ, sRing, bars, ctl};
+                M mma{tmem, sQ, sRing, bars, sched, ctl};
                 mma.init_descs();
                 mma.run(p);
                 // all MMAs issued by this warp must finish before TMEM is released
@@ -788,7 +909,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
             __syncwarp();
         } else if (warp == C::CTRL_WARP + 1) {
             if (lane == 0) {
-                FwdLoad<D, BF16> ld{&tmQ, &tmK, &tmV, sQ, sRing, bars, ctl};
+                FwdLoad<D, BF16> ld{&tmQ, &tmK, &tmV, sQ, sRing, bars, sched, ctl};
                 ld.run(p);
                 ld.drain();
             }

@@ -385,6 +385,39 @@ __device__ __forceinline__ void tmem_ld128_split(uint32_t taddr, uint32_t (&r)[1
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------------
+// Cluster launch control (sm_100): ask the hardware to cancel the launch of a CTA of
+// this grid that has not started yet.  The 16-byte response lands in shared memory
+// (16-byte aligned) and completes 16 transaction bytes on the mbarrier; the caller
+// arms the barrier with mbar_arrive_expect_tx(bar, 16) first.  After a response
+// that reports no cancellation the CTA must not ask again.
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar)
+{
+    asm volatile(
+        "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+            resp),
+        "r"(bar)
+        : "memory");
+}
+
+// Decodes a response: true and the cancelled CTA's blockIdx.x, or false.
+__device__ __forceinline__ bool clc_query(uint32_t resp, int& ctaid_x)
+{
+    uint32_t ok, x;
+    asm volatile(
+        "{\n\t.reg .b128 r;\n\t.reg .pred p;\n\t"
+        "ld.shared.b128 r, [%2];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t"
+        "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+        : "=r"(ok), "=r"(x)
+        : "r"(resp)
+        : "memory");
+    ctaid_x = static_cast<int>(x);
+    return ok != 0;
+}
+
+// ---------------------------------------------------------------------------------
 // Special-function exp2 (hardware approximation instruction).
 // ---------------------------------------------------------------------------------
 __device__ __forceinline__ float ex2_sfu(float x)

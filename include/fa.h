@@ -181,6 +181,23 @@ fa_status fa_last_device_status(fa_stream stream, uint32_t* detail);
 fa_status fa_clear_device_status(fa_stream stream);
 
 /*
+ * Order in which the forward's CTAs take their work units ("[RFC] FA4 --
+ * head_dim=256 & head_dim=512", Phase 2 "Persistent + cluster-aware tile
+ * scheduler" and Phase 3 short-sequence tuning, CLC scheduling):
+ *   FA_SCHED_STATIC (0, the default): a persistent grid of at most one CTA per SM
+ *     walks the units with a fixed stride (longest units first under the causal
+ *     mask, heads grouped so that concurrent CTAs share K/V in L2);
+ *   FA_SCHED_CLC (1): when there are more units than SMs, one CTA per unit is
+ *     launched and every running CTA takes the next unit by cancelling the launch
+ *     of a CTA that has not started (cluster launch control), in unit order.
+ * Process-wide; affects launches made after the call.  Results are identical in
+ * both modes.  Any other mode returns FA_ERR_INVALID_ARG.
+ */
+#define FA_SCHED_STATIC 0
+#define FA_SCHED_CLC 1
+fa_status fa_set_unit_schedule(int mode);
+
+/*
  * Test hook: when `mode` is 1, the next forward launch withholds its first K
  * tile copy so that the consumer's bounded wait runs out and the kernel reports
  * FA_ERR_DEVICE_TIMEOUT instead of hanging.  The hook disarms itself after one
