@@ -57,6 +57,8 @@ CASES = [
     (1, 23, 9, 2, 1, 8, True),      # Sq > Sk: the first rows see no key
     (2, 40, 31, 2, 2, 32, False),
     (1, 64, 64, 2, 2, 128, True),
+    (1, 40, 50, 4, 2, 192, True),   # the library's head dims 192 and 256
+    (1, 24, 24, 2, 2, 256, False),
 ]
 
 
