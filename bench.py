@@ -41,16 +41,41 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
-def kernel_source_digest():
-    """sha256 over the CUDA sources, to tell whether a recorded ncu capture still
-    describes the kernels that run."""
+def _strip_comments(src):
+    """C/C++ source without comments, whitespace runs collapsed (string and character
+    literals kept as written), so that a comment-only edit keeps the digest."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def kernel_source_digest(csrc=None):
+    """sha256 over the CUDA sources with comments and layout removed, to tell whether a
+    recorded ncu capture still describes the kernels that run."""
     import hashlib
-    csrc = os.path.join(ROOT, "exact_attention_blackwell_fa_b200", "csrc")
+    csrc = csrc or os.path.join(ROOT, "exact_attention_blackwell_fa_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                h.update(name.encode() + b"\0" + _strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

@@ -10,10 +10,12 @@
 //   * persistent CTAs (one per SM) walk a static list of work units
 //     (batch, query head, block of query rows); units are grouped by heads so that the
 //     CTAs running at the same time share K/V through L2, and for the causal mask the
-//     longest units (last query blocks) go first;
-//   * one TMA warp stages Q once per unit and streams K and V through a 5-deep ring
-//     of 32-KB shared-memory chunks (128 rows x 128 head-dim columns, 128-byte
-//     swizzle) guarded by full/empty mbarriers;
+//     longest units (last query blocks) go first.  Optionally (FwdParams::clc) one CTA
+//     is launched per unit and the running CTAs take the others in the same order by
+//     cluster launch control;
+//   * one TMA thread stages Q once per unit and streams K and V through a ring of
+//     shared-memory chunks (128 rows x 128 head dims, 32 KB, at d = 128 and 256; 128
+//     x 64, 16 KB, at d = 192; 128-byte swizzle) guarded by full/empty mbarriers;
 //   * one MMA warp issues tcgen05.mma: S = Q K^T into TMEM, then O += P V with P read
 //     back from TMEM (P overwrites the first half of its own S buffer as 16-bit
 //     pairs);
@@ -27,8 +29,11 @@
 //
 // head_dim 128: two Q tiles (256 query rows) per unit, TMEM = S0 | S1 | O0 | O1; the
 // tensor core alternates between the two tiles so that one tile's softmax overlaps
-// the other tile's MMAs.  head_dim 256: one Q tile, TMEM = S(a) | S(b) | O (256
-// columns), S double buffered so the next S = Q K^T runs during the softmax.
+// the other tile's MMAs; 384 threads, the control warpgroup handing registers to the
+// softmax warpgroups (setmaxnreg).  head_dim 192 / 256: one Q tile,
+// TMEM = S(a) | S(b) | O (192 / 256 columns), S double buffered so the next
+// S = Q K^T runs during the softmax; each ring chunk is waited for right before and
+// released right after the MMAs that read it.
 #pragma once
 
 #include <type_traits>

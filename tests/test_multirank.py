@@ -40,7 +40,7 @@ def _worker(rank, world, port, out):
 def test_two_replicas_max_over_ranks():
     world = 2
     port = _free_port()
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()  # no fork of a process that may hold CUDA state
     out = manager.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     assert out[0][0] == out[1][0] == 15.0
