@@ -313,8 +313,10 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     return fwd_common(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, d, causal, scale, dt, 1, nullptr, stream);
 }
 
-// Slices for the split-KV forward: enough units to cover the SMs, at least two KV
-// tiles per slice, at most 64 slices.
+// Slices for the split-KV forward: the count that minimises (waves of units over the
+// SMs) x (KV tiles per slice + a per-unit fixed cost of about two tiles: pipeline
+// fill and drain, epilogue, its share of the combine), from 1 to 64 slices of at
+// least two tiles each.  A count that leaves a short last wave costs a whole wave.
 static int splitkv_auto(int B, int Sq, int Sk, int Hq, int Hkv, int d, int sm_count)
 {
     const int group = Hq / Hkv;
@@ -322,10 +324,18 @@ static int splitkv_auto(int B, int Sq, int Sk, int Hq, int Hkv, int d, int sm_co
     const int unit = fwd_unit_rows(d);
     const long long units = (long long)B * (pack > 1 ? Hkv : Hq) * ((Sq * pack + unit - 1) / unit);
     const int nk = (Sk + 127) / 128;
-    long long s = (sm_count + units - 1) / units;
-    if (s > nk / 2) s = nk / 2;
-    if (s > 64) s = 64;
-    return s < 1 ? 1 : (int)s;
+    const int smax = nk / 2 < 64 ? nk / 2 : 64;
+    int best = 1;
+    long long best_cost = -1;
+    for (int s = 1; s <= (smax > 1 ? smax : 1); ++s) {
+        const long long waves = (units * s + sm_count - 1) / sm_count;
+        const long long cost = waves * ((nk + s - 1) / s + 2);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
 }
 
 size_t fa_fwd_splitkv_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int d, int num_splits)
