@@ -25,7 +25,7 @@
 //     grew by more than kRescaleTau (log2 units), write P back into TMEM as 16-bit
 //     pairs, and finally normalise and write O and LSE.  The exp2 can be split
 //     between the SFU and an FMA-pipe cubic (FwdCfg::POLY_EVERY); on sm_100 the SFU
-//     alone measured faster for both head dims, so the split is off;
+//     alone measured faster at every head dim, so the split is off;
 //
 // head_dim 128: two Q tiles (256 query rows) per unit, TMEM = S0 | S1 | O0 | O1; the
 // tensor core alternates between the two tiles so that one tile's softmax overlaps

@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 FA_ERR_DEVICE_TIMEOUT = 4
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [128, 192, 256])
 def test_withheld_tile_reports_timeout_then_recovers(oracle_mod, d):
     import exact_attention_blackwell_fa_b200 as fa
 
