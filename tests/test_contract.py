@@ -116,7 +116,7 @@ def test_workspace_size(lib):
         rows = B * Hq * ((Sq + 127) // 128 * 128)
         return 2 * r256(rows * 4) + r256(rows * d * 4)
 
-    for args in [(1, 1, 1, 128), (2, 16384, 16, 128), (1, 257, 8, 256), (3, 129, 5, 128)]:
+    for args in [(1, 1, 1, 128), (2, 16384, 16, 128), (1, 257, 8, 256), (3, 129, 5, 128), (2, 300, 4, 192)]:
         assert lib.fa_bwd_workspace_size(*args) == expect(*args)
     assert lib.fa_bwd_workspace_size(0, 10, 1, 128) == 0
 
