@@ -37,6 +37,7 @@ SIGNATURES = {
     "fa_clear_device_status": (_ci, [_vp]),
     "fa_debug_inject": (_ci, [_ci]),
     "fa_set_unit_schedule": (_ci, [_ci]),
+    "fa_set_exp2_emulation": (_ci, [_ci]),
     "fa_debug_exp2": (_ci, [_vp, _vp, _ci, _ci, _vp]),
 }
 

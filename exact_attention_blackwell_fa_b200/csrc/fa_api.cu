@@ -89,7 +89,7 @@ fa_status check_common(int B, int Sq, int Sk, int Hq, int Hkv, int d, float scal
     if (B < 1 || Sq < 1 || Sk < 1 || Hq < 1 || Hkv < 1) return FA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
-    if (d != 128 && d != 192 && d != 256) return FA_ERR_UNSUPPORTED;
+    if (d != 128 && d != 192 && d != 256 && d != 384 && d != 512) return FA_ERR_UNSUPPORTED;
     if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_UNSUPPORTED;
     // element counts must stay inside the 32-bit row indices the kernels use
     const long long rows_q = (long long)B * Sq * Hq, rows_k = (long long)B * Sk * Hkv;
@@ -131,6 +131,7 @@ fa_status check_regs(K kernel, int launch_regs)
 int g_inject = 0;
 std::mutex g_inject_mu;
 std::atomic<int> g_schedule{FA_SCHED_STATIC};
+std::atomic<int> g_exp2_emu{-1};  // -1: the per-head-dim default
 
 int take_inject()
 {
@@ -182,26 +183,50 @@ fa_status launch_bwd_wide(const CUtensorMap& tq, const CUtensorMap& tk64, const 
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, int EMU>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      fa::FwdParams p, int sm_count, cudaStream_t stream)
 {
     using C = fa::FwdCfg<D, BF16>;
     if constexpr (C::REG_SPLIT) {
-        static const fa_status regs_ok = check_regs(fa::fa_fwd_kernel<D, BF16>, C::REG_LAUNCH);
+        static const fa_status regs_ok = check_regs(fa::fa_fwd_kernel<D, BF16, EMU>, C::REG_LAUNCH);
         if (regs_ok != FA_OK) return regs_ok;
     }
-    fa_status st = set_smem(fa::fa_fwd_kernel<D, BF16>, C::SMEM_BYTES);
+    fa_status st = set_smem(fa::fa_fwd_kernel<D, BF16, EMU>, C::SMEM_BYTES);
     if (st != FA_OK) return st;
 
     // cluster launch control: one CTA per unit, the running ones take the rest
     const int grid = p.clc ? p.num_tiles : (p.num_tiles < sm_count ? p.num_tiles : sm_count);
-    fa::fa_fwd_kernel<D, BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    fa::fa_fwd_kernel<D, BF16, EMU><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 // query rows per forward work unit: two 128-row Q tiles at head_dim 128, one otherwise
 int fwd_unit_rows(int d) { return d == 128 ? 256 : 128; }
+
+// forward work units per Q tile: head dims 384 and 512 split V / O into two halves
+int fwd_vparts(int d) { return d > 256 ? 2 : 1; }
+
+// Exponential pairs of every four that the forward computes with the FMA-pipe cubic
+// when the caller has not chosen (fa_set_exp2_emulation(-1)), per head dim.
+int exp2_emulation_default(int d)
+{
+    (void)d;
+    return 0;
+}
+
+template <int D, bool BF16>
+fa_status launch_fwd_emu(int emu, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const fa::FwdParams& p, int sm_count, cudaStream_t s)
+{
+    switch (emu) {
+    case 0: return launch_fwd<D, BF16, 0>(tq, tk, tv, p, sm_count, s);
+    case 1: return launch_fwd<D, BF16, 1>(tq, tk, tv, p, sm_count, s);
+    case 2: return launch_fwd<D, BF16, 2>(tq, tk, tv, p, sm_count, s);
+    case 3: return launch_fwd<D, BF16, 3>(tq, tk, tv, p, sm_count, s);
+    default: return FA_ERR_INVALID_ARG;
+    }
+}
 
 fa_status launch_fwd_any(int d, bool bf16, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          fa::FwdParams p, int sm_count, cudaStream_t s)
@@ -209,10 +234,19 @@ fa_status launch_fwd_any(int d, bool bf16, const CUtensorMap& tq, const CUtensor
     // dynamic unit order (cluster launch control) when selected and there are more
     // units than SMs
     p.clc = (g_schedule.load(std::memory_order_relaxed) == FA_SCHED_CLC && p.num_tiles > sm_count) ? 1 : 0;
+    int emu = g_exp2_emu.load(std::memory_order_relaxed);
+    if (emu < 0) emu = exp2_emulation_default(d);
     switch (d) {
-    case 128: return bf16 ? launch_fwd<128, true>(tq, tk, tv, p, sm_count, s) : launch_fwd<128, false>(tq, tk, tv, p, sm_count, s);
-    case 192: return bf16 ? launch_fwd<192, true>(tq, tk, tv, p, sm_count, s) : launch_fwd<192, false>(tq, tk, tv, p, sm_count, s);
-    case 256: return bf16 ? launch_fwd<256, true>(tq, tk, tv, p, sm_count, s) : launch_fwd<256, false>(tq, tk, tv, p, sm_count, s);
+    case 128: return bf16 ? launch_fwd_emu<128, true>(emu, tq, tk, tv, p, sm_count, s)
+                          : launch_fwd_emu<128, false>(emu, tq, tk, tv, p, sm_count, s);
+    case 192: return bf16 ? launch_fwd_emu<192, true>(emu, tq, tk, tv, p, sm_count, s)
+                          : launch_fwd_emu<192, false>(emu, tq, tk, tv, p, sm_count, s);
+    case 256: return bf16 ? launch_fwd_emu<256, true>(emu, tq, tk, tv, p, sm_count, s)
+                          : launch_fwd_emu<256, false>(emu, tq, tk, tv, p, sm_count, s);
+    case 384: return bf16 ? launch_fwd_emu<384, true>(emu, tq, tk, tv, p, sm_count, s)
+                          : launch_fwd_emu<384, false>(emu, tq, tk, tv, p, sm_count, s);
+    case 512: return bf16 ? launch_fwd_emu<512, true>(emu, tq, tk, tv, p, sm_count, s)
+                          : launch_fwd_emu<512, false>(emu, tq, tk, tv, p, sm_count, s);
     default: return FA_ERR_UNSUPPORTED;
     }
 }
@@ -290,7 +324,7 @@ static fa_status fwd_common(const void* q, const void* k, const void* v, void* o
     p.group = Hq / Hkv;
     const int unit = fwd_unit_rows(d);
     p.num_m = (Sq * pack + unit - 1) / unit;
-    p.num_tiles = B * (pack > 1 ? Hkv : Hq) * p.num_m * splits;
+    p.num_tiles = B * (pack > 1 ? Hkv : Hq) * p.num_m * fwd_vparts(d) * splits;
     p.chunk_heads = pack > 1 ? chunk_heads_for(B, Hkv, 1, Sk, d) : chunk_heads_for(B, Hq, p.group, Sk, d);
     p.causal = causal ? 1 : 0;
     p.inject = take_inject();
@@ -302,7 +336,9 @@ static fa_status fwd_common(const void* q, const void* k, const void* v, void* o
     const unsigned blocks = (unsigned)((rows + 7) / 8);
     if (d == 128) launch_combine<128>(bf16, p, blocks, s);
     else if (d == 192) launch_combine<192>(bf16, p, blocks, s);
-    else launch_combine<256>(bf16, p, blocks, s);
+    else if (d == 256) launch_combine<256>(bf16, p, blocks, s);
+    else if (d == 384) launch_combine<384>(bf16, p, blocks, s);
+    else launch_combine<512>(bf16, p, blocks, s);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -322,7 +358,8 @@ static int splitkv_auto(int B, int Sq, int Sk, int Hq, int Hkv, int d, int sm_co
     const int group = Hq / Hkv;
     const int pack = (group > 1 && group <= 16 && (group & (group - 1)) == 0 && Sq < 256) ? group : 1;
     const int unit = fwd_unit_rows(d);
-    const long long units = (long long)B * (pack > 1 ? Hkv : Hq) * ((Sq * pack + unit - 1) / unit);
+    const long long units =
+        (long long)B * (pack > 1 ? Hkv : Hq) * ((Sq * pack + unit - 1) / unit) * fwd_vparts(d);
     const int nk = (Sk + 127) / 128;
     const int smax = nk / 2 < 64 ? nk / 2 : 64;
     int best = 1;
@@ -340,7 +377,9 @@ static int splitkv_auto(int B, int Sq, int Sk, int Hq, int Hkv, int d, int sm_co
 
 size_t fa_fwd_splitkv_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int d, int num_splits)
 {
-    if (B < 1 || Sq < 1 || Sk < 1 || Hq < 1 || Hkv < 1 || (d != 128 && d != 192 && d != 256) || Hq % Hkv) return 0;
+    if (B < 1 || Sq < 1 || Sk < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv ||
+        (d != 128 && d != 192 && d != 256 && d != 384 && d != 512))
+        return 0;
     if (num_splits <= 0) {
         DeviceInfo di;
         if (device_info(&di) != FA_OK) return 0;
@@ -412,7 +451,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
     p.group = Hq / Hkv;
     const int unit = fwd_unit_rows(d);
     p.num_m = (max_seqlen_q + unit - 1) / unit;
-    p.num_tiles = B * Hq * p.num_m;
+    p.num_tiles = B * Hq * p.num_m * fwd_vparts(d);
     p.chunk_heads = chunk_heads_for(B, Hq, p.group, max_seqlen_k, d);
     p.causal = causal ? 1 : 0;
     p.inject = take_inject();
@@ -439,6 +478,7 @@ static fa_status bwd_common(const void* q, const void* k, const void* v, const v
         return FA_ERR_INVALID_ARG;
     fa_status st = check_common(B, Sq, Sk, Hq, Hkv, d, scale, dt);
     if (st != FA_OK) return st;
+    if (d > 256) return FA_ERR_UNSUPPORTED;  // the backward covers head dims up to 256
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
         !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -580,6 +620,13 @@ fa_status fa_set_unit_schedule(int mode)
     return FA_OK;
 }
 
+fa_status fa_set_exp2_emulation(int pairs_of_4)
+{
+    if (pairs_of_4 < -1 || pairs_of_4 > 3) return FA_ERR_INVALID_ARG;
+    g_exp2_emu.store(pairs_of_4, std::memory_order_relaxed);
+    return FA_OK;
+}
+
 fa_status fa_debug_inject(int mode)
 {
     if (mode != 0 && mode != 1) return FA_ERR_INVALID_ARG;
@@ -629,6 +676,7 @@ extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
 {
     fa_status st = check_common(B, Sq, Sk, Hq, Hkv, d, scale, dt);
     if (st != FA_OK) return st;
+    if (d > 256) return FA_ERR_UNSUPPORTED;
     if (fa::bwd_workspace_bytes(B, Sq, Hq, d) > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_SCRATCH_LIMIT;
     void* scratch = nullptr;
     st = noalloc_scratch(&scratch);

@@ -23,9 +23,10 @@
 //     columns of a tile in registers) loads S from TMEM, applies the scale and
 //     mask, keep the running row max and sum, rescale O in TMEM only when the row max
 //     grew by more than kRescaleTau (log2 units), write P back into TMEM as 16-bit
-//     pairs, and finally normalise and write O and LSE.  The exp2 can be split
-//     between the SFU and an FMA-pipe cubic (FwdCfg::POLY_EVERY); on sm_100 the SFU
-//     alone measured faster at every head dim, so the split is off;
+//     pairs, and finally normalise and write O and LSE.  The exp2 of tiles that need
+//     no mask can be split between the SFU and an FMA-pipe cubic: EMU of every four
+//     pairs of exponentials on the FMA pipe (template parameter, chosen per call by
+//     the host; 0 keeps every exponential on the SFU);
 //
 // head_dim 128: two Q tiles (256 query rows) per unit, TMEM = S0 | S1 | O0 | O1; the
 // tensor core alternates between the two tiles so that one tile's softmax overlaps
@@ -33,7 +34,12 @@
 // softmax warpgroups (setmaxnreg).  head_dim 192 / 256: one Q tile,
 // TMEM = S(a) | S(b) | O (192 / 256 columns), S double buffered so the next
 // S = Q K^T runs during the softmax; each ring chunk is waited for right before and
-// released right after the MMAs that read it.
+// released right after the MMAs that read it.  head_dim 384 / 512 ("[RFC] FA4 --
+// head_dim=256 & head_dim=512", Phase 4): the same one-tile pipeline, but a row's
+// fp32 O no longer fits beside two S buffers, so each Q tile is two units, each
+// covering one half of V's and O's head dims (TMEM = S(a) | S(b) | O half) and
+// computing S = Q K^T over all of them; both units see the same scores and row
+// statistics, and the first writes the LSE.
 #pragma once
 
 #include <type_traits>
@@ -91,20 +97,26 @@ enum : uint32_t {
 
 template <int D, bool BF16>
 struct FwdCfg {
-    static_assert(D == 128 || D == 192 || D == 256, "head_dim");
+    static_assert(D == 128 || D == 192 || D == 256 || D == 384 || D == 512, "head_dim");
     static constexpr int NQ = D == 128 ? 2 : 1;  // 128-row Q tiles per work unit
     static constexpr int NS = D == 128 ? 1 : 2;  // S buffers per Q tile
+    // head dims of V and O a unit covers: all of them up to 256; at 384 and 512 the
+    // fp32 O accumulator of a whole row (D TMEM columns) does not fit beside two S
+    // buffers, so a unit covers one half of V / O (NPASS = 2 units per Q tile, each
+    // recomputing S = Q K^T over all D dims)
+    static constexpr int DV = D > 256 ? D / 2 : D;
+    static constexpr int NPASS = D / DV;
     // ring chunk: 128 rows x CHUNK_COLS head dims (one or two 64-column swizzle atoms).
-    // With one Q tile (d = 192, 256) each chunk is waited for just before and released
+    // With one Q tile (d >= 192) each chunk is waited for just before and released
     // just after the MMAs that read it, so the ring refills while the rest of the tile
     // is still being read
-    static constexpr int CHUNK_COLS = D == 192 ? 64 : 128;
-    static constexpr int KCH = D / CHUNK_COLS;    // chunks per K (or V) tile
-    static constexpr int NSTAGE = D == 192 ? 11 : 5;  // ring depth, in chunks
+    static constexpr int CHUNK_COLS = (D == 128 || D == 256) ? 128 : 64;
+    static constexpr int KCH = D / CHUNK_COLS;    // chunks per K tile
+    static constexpr int VCH = DV / CHUNK_COLS;   // chunks per V tile (the unit's part)
+    // ring depth, in chunks: what shared memory leaves beside the Q tile
+    static constexpr int NSTAGE = D == 192 ? 11 : D == 384 ? 8 : D == 512 ? 6 : 5;
     static constexpr int BM = 128;               // query rows per Q tile
     static constexpr int BN = 128;               // keys per KV tile
-    static constexpr int POLY_EVERY = 0;         // exp2 pairs: 1 in POLY_EVERY on the FMA pipe (0: none)
-    static constexpr int POLY_MOD = POLY_EVERY > 0 ? POLY_EVERY : 1;
     // spinning waits (see fa_common.cuh) for the softmax and MMA warps
     static constexpr bool SPIN = D == 128;
     static constexpr int UNIT_ROWS = NQ * BM;
@@ -166,10 +178,12 @@ struct FwdCfg {
     static constexpr uint32_t IDESC_PV = idesc_f16(BF16, 128, CHUNK_COLS, false, true);
 };
 
-template <int UNIT_ROWS>
-__device__ __forceinline__ void fwd_decode(const FwdParams& p, int t, int& b, int& h, int& m0)
+template <int UNIT_ROWS, int NPASS>
+__device__ __forceinline__ void fwd_decode(const FwdParams& p, int t, int& b, int& h, int& m0, int& vpass)
 {
     t /= p.splits;  // the slices of one unit are adjacent in the list
+    vpass = t % NPASS;  // then the V / O parts of one Q tile
+    t /= NPASS;
     const int H = p.pack > 1 ? p.Hkv : p.Hq;  // heads of the unit list
     const int BH = p.B * H;
     const int per_chunk = p.chunk_heads * p.num_m;
@@ -196,14 +210,15 @@ struct FwdUnit {
     int n;                 // KV tiles to visit: j0 .. j0 + n - 1
     int j0;                // first KV tile (split KV: the slice's first)
     int split;             // slice index (split KV), else 0
+    int vpass;             // which part of V / O's head dims (head_dim > 256), else 0
     bool rows;             // the unit has query rows at all
 };
 
-template <int UNIT_ROWS>
+template <int UNIT_ROWS, int NPASS>
 __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int t)
 {
     FwdUnit u;
-    fwd_decode<UNIT_ROWS>(p, t, u.b, u.h, u.m0);
+    fwd_decode<UNIT_ROWS, NPASS>(p, t, u.b, u.h, u.m0, u.vpass);
     if (p.cu_q != nullptr) {
         u.tb = 0;
         u.q_base = p.cu_q[u.b];
@@ -296,7 +311,31 @@ struct FwdUnits {
 // Softmax / epilogue warpgroup, one per 128-row Q tile: thread = one query row, all
 // 128 key columns of a tile held in registers.
 // ---------------------------------------------------------------------------------
-template <int D, bool BF16>
+// P = 2^x for the 32 columns cc*32 .. cc*32+31 of a tile row, packed to 16-bit pairs,
+// with the row-sum partials accumulated.  SPLIT: pair j of the row goes to the FMA-pipe
+// cubic when (j mod 4) < EMU, else to the SFU.
+template <bool BF16, int EMU, bool SPLIT>
+__device__ __forceinline__ void fwd_exp_block(const uint32_t (&sr)[128], int cc, uint64_t sl2x2, uint64_t negm2,
+                                              uint64_t (&acc2)[2], uint32_t (&pk)[16])
+{
+#pragma unroll
+    for (int k = 0; k < 32; k += 2) {
+        const int c = cc * 32 + k;
+        const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm2);
+        float e0, e1;
+        if (SPLIT && ((c >> 1) & 3) < EMU) {
+            exp2_fma_x2(x2, e0, e1);
+        } else {
+            const float2 x = f2unpack(x2);
+            e0 = ex2_sfu(x.x);
+            e1 = ex2_sfu(x.y);
+        }
+        acc2[(k >> 1) & 1] = fadd2(acc2[(k >> 1) & 1], f2pack(e0, e1));
+        pk[k >> 1] = pack2_p<BF16>(e0, e1);
+    }
+}
+
+template <int D, bool BF16, int EMU>
 __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars, uint32_t sched, CtaCtl* ctl, int q,
                                 int wq)
 {
@@ -312,7 +351,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
 
     FwdUnits<D, BF16, true> units{bars, sched, ctl, p.clc};
     for (int t = units.first(p); t >= 0; t = units.next(p)) {
-        const FwdUnit u = fwd_unit<C::UNIT_ROWS>(p, t);
+        const FwdUnit u = fwd_unit<C::UNIT_ROWS, C::NPASS>(p, t);
         if (!u.rows) continue;  // past the end of its (shorter) sequence: nothing to do
         const int n = u.n;
         const int vr = u.m0 + q * C::BM + r_in_tile;  // this thread's row in the unit's row space
@@ -321,16 +360,20 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
         const int q0 = (u.m0 + q * C::BM) / p.pack;   // the Q tile's first (smallest) query
         const bool row_ok = vr < u.R;
         const size_t orow_idx = static_cast<size_t>(u.tb) * p.Sq_alloc + u.q_base + row;
-        T* orow = reinterpret_cast<T*>(p.o) + (orow_idx * p.Hq + h) * D;
+        // this unit's part of the O row (all of it up to head_dim 256)
+        T* orow = reinterpret_cast<T*>(p.o) + (orow_idx * p.Hq + h) * D + u.vpass * C::DV;
         float* lrow = p.lse + (static_cast<size_t>(u.tb) * p.Hq + h) * p.Sq_alloc + u.q_base + row;
+        // the LSE is the same for every part; the first writes it
+        const bool lse_writer = u.vpass == 0;
         // split KV: this slice's partial O and LSE rows
         const size_t prow = ((static_cast<size_t>(u.split) * p.B + u.b) * p.Hq + h) * p.Sq + row;
+        float* const opart_row = p.opart + prow * D + u.vpass * C::DV;
         if (n == 0 && p.splits > 1) {  // an empty slice
             if (row_ok) {
                 const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int c = 0; c < D / 4; ++c) reinterpret_cast<float4*>(p.opart + prow * D)[c] = z;
-                p.lsepart[prow] = -INFINITY;
+                for (int c = 0; c < C::DV / 4; ++c) reinterpret_cast<float4*>(opart_row)[c] = z;
+                if (lse_writer) p.lsepart[prow] = -INFINITY;
             }
             continue;
         }
@@ -338,8 +381,8 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
             if (row_ok) {
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
-                *lrow = -INFINITY;
+                for (int c = 0; c < C::DV / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
+                if (lse_writer) *lrow = -INFINITY;
             }
             continue;
         }
@@ -397,25 +440,22 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
             const float negm = (m_ref == -INFINITY) ? 0.0f : -m_ref;
             const uint64_t negm2 = f2pack(negm, negm);
             uint64_t acc2[2] = {f2pack(0.0f, 0.0f), f2pack(0.0f, 0.0f)};
+            // masked tiles keep every exponential on the SFU, whose 2^-inf is exactly 0
+            // (the cubic's input clamp would leave 2^-126 for a masked key)
+            if (EMU > 0 && !masked) {
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int k = 0; k < 32; k += 2) {
-                    const int c = cc * 32 + k;
-                    const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm2);
-                    float e0, e1;
-                    if (C::POLY_EVERY > 0 && !masked && (c >> 1) % C::POLY_MOD == C::POLY_MOD - 1) {
-                        exp2_fma_x2(x2, e0, e1);
-                    } else {
-                        const float2 x = f2unpack(x2);
-                        e0 = ex2_sfu(x.x);
-                        e1 = ex2_sfu(x.y);
-                    }
-                    acc2[(k >> 1) & 1] = fadd2(acc2[(k >> 1) & 1], f2pack(e0, e1));
-                    pk[k >> 1] = pack2_p<BF16>(e0, e1);
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t pk[16];
+                    fwd_exp_block<BF16, EMU, true>(sr, cc, sl2x2, negm2, acc2, pk);
+                    tmem_st16(tS + cc * 16, pk);
                 }
-                tmem_st16(tS + cc * 16, pk);
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t pk[16];
+                    fwd_exp_block<BF16, EMU, false>(sr, cc, sl2x2, negm2, acc2, pk);
+                    tmem_st16(tS + cc * 16, pk);
+                }
             }
             const float2 a = f2unpack(fadd2(acc2[0], acc2[1]));
             // O must hold every earlier P V product before it is rescaled: with one S
@@ -428,7 +468,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
                     tc_fence_after();
                 }
 #pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
+                for (int cc = 0; cc < C::DV / 32; ++cc) {
                     uint32_t r[32];
                     tmem_ld32_wait(tO + cc * 32, r);
 #pragma unroll
@@ -450,23 +490,23 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
         const float lse_row = (l > 0.0f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
         if (p.splits > 1) {  // the slice's normalised O in fp32, and its LSE
 #pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
+            for (int cc = 0; cc < C::DV / 32; ++cc) {
                 uint32_t r[32];
                 tmem_ld32_wait(tO + cc * 32, r);
                 if (row_ok) {
-                    float4* dst = reinterpret_cast<float4*>(p.opart + prow * D + cc * 32);
+                    float4* dst = reinterpret_cast<float4*>(opart_row + cc * 32);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
                         dst[k] = make_float4(__uint_as_float(r[4 * k]) * inv, __uint_as_float(r[4 * k + 1]) * inv,
                                              __uint_as_float(r[4 * k + 2]) * inv, __uint_as_float(r[4 * k + 3]) * inv);
                 }
             }
-            if (row_ok) p.lsepart[prow] = lse_row;
+            if (row_ok && lse_writer) p.lsepart[prow] = lse_row;
             tc_fence_before();
             continue;
         }
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
+        for (int cc = 0; cc < C::DV / 32; ++cc) {
             uint32_t r[32];
             tmem_ld32_wait(tO + cc * 32, r);
             uint32_t pk[16];
@@ -481,7 +521,7 @@ __device__ void fwd_softmax_row(const FwdParams& p, uint32_t tmem, uint32_t bars
                 dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
             }
         }
-        if (row_ok) *lrow = lse_row;
+        if (row_ok && lse_writer) *lrow = lse_row;
         tc_fence_before();
     }
 }
@@ -556,21 +596,21 @@ struct FwdMma {
         }
         return true;
     }
-    // O_q (+)= P(q, sb) V, V tile in ring chunks sV .. sV + KCH - 1 (chunk c = O columns
-    // c*CHUNK_COLS .. (c+1)*CHUNK_COLS-1)
+    // O_q (+)= P(q, sb) V, V tile (the unit's part of its head dims) in ring chunks
+    // sV .. sV + VCH - 1 (chunk c = O columns c*CHUNK_COLS .. (c+1)*CHUNK_COLS-1)
     // (k-steps 0-3 read P of key columns 0-63, 4-7 of 64-127.)  STREAM: chunk by chunk,
     // each waited for before and released after its eight k-steps.
     template <bool STREAM>
     __device__ bool issue_PV(int q, int sb, uint32_t sV, bool acc)
     {
-        uint64_t vd[C::KCH];
+        uint64_t vd[C::VCH];
 #pragma unroll
-        for (int c = 0; c < C::KCH; ++c) vd[c] = vdesc0 + slot_off(sV + c);
+        for (int c = 0; c < C::VCH; ++c) vd[c] = vdesc0 + slot_off(sV + c);
         const uint32_t tP = tmem + C::col_S(q, sb);
         const uint32_t tO = tmem + C::col_O(q);
         if constexpr (STREAM) {
 #pragma unroll
-            for (int c = 0; c < C::KCH; ++c) {
+            for (int c = 0; c < C::VCH; ++c) {
                 if (!wait_full(sV + c)) return false;
                 tc_fence_after();
 #pragma unroll
@@ -584,7 +624,7 @@ struct FwdMma {
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t a = tP + C::col_Pk(kk);
 #pragma unroll
-                for (int c = 0; c < C::KCH; ++c)
+                for (int c = 0; c < C::VCH; ++c)
                     ts(tO + c * C::CHUNK_COLS, a, vd[c] + (kk * 2048u >> 4), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
             }
         }
@@ -608,7 +648,7 @@ struct FwdMma {
         uint32_t q_it = 0;
         FwdUnits<D, BF16, WARP_ISSUE> units{bars, sched, ctl, p.clc};
         for (int t = units.first(p); t >= 0; t = units.next(p)) {
-            const int n = fwd_unit<C::UNIT_ROWS>(p, t).n;
+            const int n = fwd_unit<C::UNIT_ROWS, C::NPASS>(p, t).n;
             if (n == 0) continue;
             if (!wait(bar(C::B_Q_FULL), q_it & 1u, W_FWD_Q_FULL)) return;
             ++q_it;
@@ -674,7 +714,7 @@ struct FwdMma {
                 if (n <= 2) commit(bar(C::B_Q_EMPTY));
                 for (int j = 0; j < n; ++j) {
                     const uint32_t sV = seq;
-                    seq += C::KCH;
+                    seq += C::VCH;
                     const int sbp = p_it[0] & 1;
                     if (!wait(bar(C::B_P_FULL + sbp), (p_it[0] >> 1) & 1u, W_FWD_P_FULL)) return;
                     tc_fence_after();
@@ -734,10 +774,11 @@ struct FwdLoad {
         filled[slot] = static_cast<int>(round);
         return true;
     }
-    __device__ bool load_kv(const CUtensorMap* tm, int row0, int hkv, int b)
+    // nch chunks of one K or V tile, head dims col0 .. col0 + nch * CHUNK_COLS - 1
+    __device__ bool load_kv(const CUtensorMap* tm, int row0, int hkv, int b, int nch, int col0)
     {
-        for (int c = 0; c < C::KCH; ++c)
-            if (!load_chunk(tm, row0, c * C::CHUNK_COLS, hkv, b)) return false;
+        for (int c = 0; c < nch; ++c)
+            if (!load_chunk(tm, row0, col0 + c * C::CHUNK_COLS, hkv, b)) return false;
         return true;
     }
 
@@ -787,7 +828,7 @@ struct FwdLoad {
     __device__ bool load_unit(const FwdParams& p, int t, uint32_t& q_it)
     {
         {
-            const FwdUnit u = fwd_unit<C::UNIT_ROWS>(p, t);
+            const FwdUnit u = fwd_unit<C::UNIT_ROWS, C::NPASS>(p, t);
             const int n = u.n, b = u.tb;
             if (n == 0) return true;
             const int hkv = p.pack > 1 ? u.h : u.h / p.group;
@@ -805,17 +846,19 @@ struct FwdLoad {
                                 u.q_base + (u.m0 + q * C::BM) / p.pack, b);
             q_round = static_cast<int>(q_it);
             ++q_it;
+            // K over all head dims; V over the unit's part of them
+            const int vcol = u.vpass * C::DV;
             if constexpr (C::NQ == 2) {
                 for (int j = 0; j < n; ++j) {
-                    if (!load_kv(tmK, krow(j), hkv, b)) return false;
-                    if (!load_kv(tmV, krow(j), hkv, b)) return false;
+                    if (!load_kv(tmK, krow(j), hkv, b, C::KCH, 0)) return false;
+                    if (!load_kv(tmV, krow(j), hkv, b, C::VCH, vcol)) return false;
                 }
             } else {
                 for (int j = 0; j < 2 && j < n; ++j)
-                    if (!load_kv(tmK, krow(j), hkv, b)) return false;
+                    if (!load_kv(tmK, krow(j), hkv, b, C::KCH, 0)) return false;
                 for (int j = 0; j < n; ++j) {
-                    if (!load_kv(tmV, krow(j), hkv, b)) return false;
-                    if (j + 2 < n && !load_kv(tmK, krow(j + 2), hkv, b)) return false;
+                    if (!load_kv(tmV, krow(j), hkv, b, C::VCH, vcol)) return false;
+                    if (j + 2 < n && !load_kv(tmK, krow(j + 2), hkv, b, C::KCH, 0)) return false;
                 }
             }
         }
@@ -835,7 +878,7 @@ struct FwdLoad {
     }
 };
 
-template <int D, bool BF16>
+template <int D, bool BF16, int EMU>
 __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p)
@@ -898,7 +941,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
 
     if (warp < C::SOFTMAX_WARPS) {
         if constexpr (C::REG_SPLIT) setmaxnreg_inc<C::REG_SOFTMAX>();  // granted once warps 8-11 released theirs
-        fwd_softmax_row<D, BF16>(p, tmem, bars, sched, ctl, warp / 4, warp & 3);
+        fwd_softmax_row<D, BF16, EMU>(p, tmem, bars, sched, ctl, warp / 4, warp & 3);
     } else {
         if constexpr (C::REG_SPLIT) setmaxnreg_dec<C::REG_CTRL>();  // every control warp, first thing
         if (warp == C::CTRL_WARP) {

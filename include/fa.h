@@ -23,10 +23,11 @@
  *     reads key/value head h / (Hq / Hkv).
  *   - causal != 0 applies a lower-triangular mask aligned to the bottom-right
  *     corner: key j is visible to query i iff j <= i + (Sk - Sq).
- *   - head_dim d must be 128, 192 or 256 (192: "[RFC] FA4 -- head_dim=256 &
- *     head_dim=512", Phase 4, symmetric head_dim=192); dtype must be FA_BF16 or
- *     FA_FP16 and is the same for every 16-bit tensor of a call.  Every pointer
- *     must be 16-byte aligned.
+ *   - head_dim d must be 128, 192, 256, 384 or 512 (192, 384, 512: "[RFC] FA4 --
+ *     head_dim=256 & head_dim=512", Phase 4, symmetric head dims; the backward
+ *     entry points take d up to 256 and return FA_ERR_UNSUPPORTED above); dtype
+ *     must be FA_BF16 or FA_FP16 and is the same for every 16-bit tensor of a call.
+ *     Every pointer must be 16-byte aligned.
  *   - Ownership: the caller owns every buffer.  The library allocates no device
  *     memory per call; scratch for the backward is the caller's workspace.
  *     Work is enqueued on `stream` and runs asynchronously; nothing synchronises.
@@ -153,6 +154,11 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
  *
  * Set-up: the first call on each device looks up the device address of the array
  * (with that device current); make that first call before any stream capture.
+ * The address is kept for the life of the process and belongs to the context that
+ * was current at that first call, the device's primary context (the one the CUDA
+ * runtime and PyTorch use).  Calls from another context on the same device (one
+ * made with cuCtxCreate), or after cudaDeviceReset, are not supported: the library
+ * is loaded into that context again and the kept address does not refer to it.
  * Every call on a device shares the one array and leaves its contents behind; the
  * kernels rewrite everything they read from it (the accumulator is zeroed by the
  * first kernel of each call), but two calls whose kernels overlap on the GPU --
@@ -165,6 +171,22 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          const float* lse, const void* dout, void* dq, void* dk, void* dv,
                          int B, int Sq, int Sk, int Hq, int Hkv, int d, int causal, float scale,
                          fa_dtype dt, fa_stream stream);
+
+/*
+ * exp2 split of the forward's softmax ("FlashAttention 4: Snellere,
+ * Geheugenefficiente Aandacht voor LLM's", section "Software-exponentials via
+ * CUDA-kernen": part of the exponentials go to a cubic polynomial on the FMA pipe
+ * instead of the special-function unit; "[RFC] FA4 -- head_dim=256 &
+ * head_dim=512", Phase 2 "exp2 FMA emulation": 3 of every 4 at head_dim 256).
+ * pairs_of_4 in 0..3 is how many of every four pairs of exponentials of a score tile
+ * use the cubic (max relative error 1.44e-4, below the 16-bit rounding of P); 0
+ * keeps every exponential on the special-function unit; -1 (the initial setting)
+ * selects the library's default for each head dim.  Tiles that need the causal or
+ * sequence-end mask always use the special-function unit.  Process-wide; affects
+ * forward launches made after the call (every forward entry point).  Any other
+ * value returns FA_ERR_INVALID_ARG.
+ */
+fa_status fa_set_exp2_emulation(int pairs_of_4);
 
 /* Static, human-readable name of a status code. */
 const char* fa_status_string(fa_status s);

@@ -40,3 +40,18 @@ def test_recorded_traffic_matches_current_sources():
         else:
             assert got is None
     assert bench.recorded_traffic("no such kernel", "no such workload") is None
+
+
+def test_choose_peak_follows_the_clock_the_kernel_ran_at():
+    peaks = {"bf16_tflops": 1606.3, "bf16_tflops_sustained": 1367.3, "sm_max_mhz": 1965.0,
+             "clocks_under_load": {"sm_mhz_median": 1305.0}}
+    p, kind, why = bench.choose_peak(peaks, {"sm_mhz": 1965.0}, 0.34)
+    assert (p, kind) == (1606.3, "burst") and "1965" in why
+    p, kind, _ = bench.choose_peak(peaks, {"sm_mhz": 1320.0}, 5.0)
+    assert (p, kind) == (1367.3, "sustained")
+    # no clock record: short regions take the burst figure, long ones the sustained
+    assert bench.choose_peak(peaks, None, 0.5)[1] == "burst"
+    assert bench.choose_peak(peaks, None, 4.0)[1] == "sustained"
+    # fallback figures when no measured file exists
+    p, kind, _ = bench.choose_peak({}, None, 0.5)
+    assert p == bench.FALLBACK_PEAKS["bf16_tflops"] and kind == "burst"

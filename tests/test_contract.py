@@ -90,8 +90,8 @@ def bwd_call(lib, **kw):
     (dict(scale=float("nan")), FA_ERR_INVALID_ARG),
     (dict(scale=float("inf")), FA_ERR_INVALID_ARG),
     (dict(d=64), FA_ERR_UNSUPPORTED),
-    (dict(d=384), FA_ERR_UNSUPPORTED),
-    (dict(d=512), FA_ERR_UNSUPPORTED),
+    (dict(d=320), FA_ERR_UNSUPPORTED),
+    (dict(d=1024), FA_ERR_UNSUPPORTED),
     (dict(dt=2), FA_ERR_UNSUPPORTED),
     (dict(q=FAKE + 2), FA_ERR_INVALID_ARG),
     (dict(v=FAKE + 8), FA_ERR_INVALID_ARG),
@@ -144,3 +144,22 @@ def test_python_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 8, 1, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fa.fa_fwd(q, q, q)
+
+
+def test_exp2_emulation_setting_validated(lib):
+    for k in (-1, 0, 1, 2, 3):
+        assert lib.fa_set_exp2_emulation(k) == FA_OK
+    for k in (-2, 4, 100):
+        assert lib.fa_set_exp2_emulation(k) == FA_ERR_INVALID_ARG
+    assert lib.fa_set_exp2_emulation(-1) == FA_OK
+
+
+def test_wide_head_dims_reach_the_device_check_forward_only(lib):
+    """head_dim 384 and 512 are valid forward arguments (the call stops at the device
+    query here, with no usable GPU); the backward refuses them before any CUDA call."""
+    import torch
+
+    for d in (384, 512):
+        assert bwd_call(lib, d=d) == FA_ERR_UNSUPPORTED
+        if not torch.cuda.is_available():
+            assert fwd_call(lib, d=d) in (FA_ERR_CUDA, FA_ERR_UNSUPPORTED)

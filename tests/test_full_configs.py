@@ -10,8 +10,9 @@ first and last query row of every head plus seeded random rows.  Shapes:
   * video-diffusion shapes [1, 257, 8, 128] (every row) and [1, 20480, 56, 128],
     inputs 0.5 N(0, 1);
   * backward: d=128, H=16, B=2, seqlen 4k/8k/16k, causal and not; d=256, H=8, B=1,
-    seqlen 16k: dQ on sampled query rows, dK/dV on sampled key rows of one KV head
-    (the oracle recomputes that head's full row statistics for them).
+    seqlen 16k: dQ on sampled query rows, dK/dV on sampled key rows of the first,
+    a middle and the last KV head of the first and last batch entries (the oracle
+    recomputes those heads' full row statistics for them).
 
 Tolerances are the parity tests': O max abs <= 1e-2 (+ half an output ulp), mean
 <= 1e-3, LSE abs <= 1e-3; gradients max abs <= 5e-2 x the largest oracle magnitude.
@@ -97,11 +98,18 @@ def _check_bwd(oracle_mod, shape, causal, seed=0):
     code, detail = fa.fa_last_device_status()
     assert code == 0, f"device status {code} ({detail:#x})"
     qrows = sample_rows(shape.B, shape.Hq, shape.Sq, 3, seed=seed + 5)
-    # dK / dV: a few key rows of the last KV head of the last batch
+    # dK / dV: key rows of several (batch entry, KV head) pairs -- the first and the
+    # last KV head, one in the middle, in the first and the last batch entry -- so that
+    # a slip in mapping key blocks to heads in the persistent, L2-grouped unit order
+    # shows up on some head: the first and last key of each plus two random ones
     g = torch.Generator().manual_seed(seed + 9)
-    js = torch.unique(torch.cat([torch.randint(0, shape.Sk, (4,), generator=g),
-                                 torch.tensor([0, shape.Sk - 1])]))
-    kvrows = torch.stack([torch.full_like(js, shape.B - 1), torch.full_like(js, shape.Hkv - 1), js], 1)
+    pairs = sorted({(0, 0), (shape.B - 1, shape.Hkv // 2), (shape.B - 1, shape.Hkv - 1), (0, shape.Hkv - 1)})
+    kv = []
+    for b_, h_ in pairs:
+        js = torch.unique(torch.cat([torch.randint(0, shape.Sk, (2,), generator=g),
+                                     torch.tensor([0, shape.Sk - 1])]))
+        kv.append(torch.stack([torch.full_like(js, b_), torch.full_like(js, h_), js], 1))
+    kvrows = torch.cat(kv)
     rq, rk, rv, _ = oracle_mod.bwd(q, k, v, do, causal=causal, qrows=qrows, kvrows=kvrows)
     b, h, i = qrows[:, 0], qrows[:, 1], qrows[:, 2]
     got_q = dq[b.cuda(), i.cuda(), h.cuda()].cpu().double()

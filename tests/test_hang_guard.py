@@ -43,4 +43,10 @@ def test_withheld_tile_reports_timeout_then_recovers(oracle_mod, d):
     torch.cuda.synchronize()
     assert fa.fa_last_device_status()[0] == 0
     o_ref, _ = oracle_mod.fwd(q, k, v)
-    assert (o.cpu().double() - o_ref).abs().max().item() <= 1.2e-2
+    # the forward parity bound: max abs 1e-2 over the value before its own rounding to
+    # bf16 (so half an output ulp on top), mean abs 1e-3
+    err = (o.cpu().double() - o_ref).abs()
+    e = torch.floor(torch.log2(o_ref.abs().clamp_min(torch.finfo(torch.bfloat16).tiny)))
+    half_ulp = torch.ldexp(torch.ones_like(o_ref), (e - 8).to(torch.int32))
+    assert (err - (1e-2 + half_ulp)).max().item() <= 0.0, err.max().item()
+    assert err.mean().item() <= 1e-3

@@ -30,11 +30,12 @@ def test_splitkv_workspace_size(lib):
     # float32 partial O and LSE per slice and row, each part rounded to 256 bytes
     r256 = lambda x: (x + 255) // 256 * 256
     for (B, Sq, Sk, Hq, Hkv, d, s) in [(2, 1, 4096, 16, 2, 128, 8), (1, 7, 100, 4, 4, 256, 3),
-                                       (3, 5, 1000, 8, 2, 192, 4)]:
+                                       (3, 5, 1000, 8, 2, 192, 4), (1, 3, 900, 4, 2, 512, 3),
+                                       (2, 2, 700, 2, 1, 384, 2)]:
         rows = s * B * Hq * Sq
         assert lib.fa_fwd_splitkv_workspace_size(B, Sq, Sk, Hq, Hkv, d, s) == r256(rows * d * 4) + r256(rows * 4)
     assert lib.fa_fwd_splitkv_workspace_size(1, 1, 1, 3, 2, 128, 2) == 0   # Hq % Hkv
-    assert lib.fa_fwd_splitkv_workspace_size(1, 1, 1, 2, 2, 384, 2) == 0   # head dim
+    assert lib.fa_fwd_splitkv_workspace_size(1, 1, 1, 2, 2, 320, 2) == 0   # head dim
 
 
 def test_splitkv_rejections(lib):

@@ -44,7 +44,7 @@ def varlen_call(lib, **kw):
     (dict(B=0), FA_ERR_INVALID_ARG),
     (dict(mq=0), FA_ERR_INVALID_ARG),
     (dict(Hq=3, Hkv=2), FA_ERR_INVALID_ARG),
-    (dict(d=384), FA_ERR_UNSUPPORTED),
+    (dict(d=320), FA_ERR_UNSUPPORTED),
     (dict(q=None), FA_ERR_INVALID_ARG),
     (dict(o=FAKE + 8), FA_ERR_INVALID_ARG),
 ])
