@@ -478,7 +478,6 @@ static fa_status bwd_common(const void* q, const void* k, const void* v, const v
         return FA_ERR_INVALID_ARG;
     fa_status st = check_common(B, Sq, Sk, Hq, Hkv, d, scale, dt);
     if (st != FA_OK) return st;
-    if (d > 256) return FA_ERR_UNSUPPORTED;  // the backward covers head dims up to 256
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
         !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -520,7 +519,8 @@ static fa_status bwd_common(const void* q, const void* k, const void* v, const v
     p.Sq_pad = (int)sq_pad;
     p.num_n = (Sk + kv_rows - 1) / kv_rows;
     p.num_m = (Sq + 127) / 128;
-    p.num_units = B * Hkv * p.num_n;
+    // head dims 384 / 512: each key block is two units, one per half of the output dims
+    p.num_units = B * Hkv * p.num_n * (d > 256 ? 2 : 1);
     // KV heads whose Q and dO streams stay inside L2 together
     {
         const double qdo_bytes = 2.0 * Sq * d * 2.0 * p.group;
@@ -533,6 +533,12 @@ static fa_status bwd_common(const void* q, const void* k, const void* v, const v
     p.scale = scale;
     p.sl2 = scale * 1.4426950408889634f;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 512)
+        return bf16 ? launch_bwd_wide<512, true>(tq, tk, tv, tdo, p, di.sm_count, s)
+                    : launch_bwd_wide<512, false>(tq, tk, tv, tdo, p, di.sm_count, s);
+    if (d == 384)
+        return bf16 ? launch_bwd_wide<384, true>(tq, tk, tv, tdo, p, di.sm_count, s)
+                    : launch_bwd_wide<384, false>(tq, tk, tv, tdo, p, di.sm_count, s);
     if (d == 256)
         return bf16 ? launch_bwd_wide<256, true>(tq, tk, tv, tdo, p, di.sm_count, s)
                     : launch_bwd_wide<256, false>(tq, tk, tv, tdo, p, di.sm_count, s);
@@ -676,7 +682,6 @@ extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
 {
     fa_status st = check_common(B, Sq, Sk, Hq, Hkv, d, scale, dt);
     if (st != FA_OK) return st;
-    if (d > 256) return FA_ERR_UNSUPPORTED;
     if (fa::bwd_workspace_bytes(B, Sq, Hq, d) > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_SCRATCH_LIMIT;
     void* scratch = nullptr;
     st = noalloc_scratch(&scratch);

@@ -122,21 +122,29 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p)
         const size_t off = (trow * p.Hq + h) * D + lane * (D / 32);
         constexpr int NW = D / 64;  // 32-bit words per lane (two 16-bit values each)
         uint32_t ow[NW], dw[NW];
+        const uint16_t* o16 = static_cast<const uint16_t*>(p.o) + off;
+        const uint16_t* d16 = static_cast<const uint16_t*>(p.dout) + off;
         if constexpr (NW == 3) {  // 12 bytes per lane: 4-byte aligned only
 #pragma unroll
             for (int w = 0; w < NW; ++w) {
-                ow[w] = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.o) + off)[w];
-                dw[w] = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.dout) + off)[w];
+                ow[w] = reinterpret_cast<const uint32_t*>(o16)[w];
+                dw[w] = reinterpret_cast<const uint32_t*>(d16)[w];
             }
-        } else if constexpr (NW == 2) {
-            const uint2 a = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.o) + off);
-            const uint2 c = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.dout) + off);
-            ow[0] = a.x; ow[1] = a.y; dw[0] = c.x; dw[1] = c.y;
-        } else {
-            const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + off);
-            const uint4 c = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + off);
-            ow[0] = a.x; ow[1] = a.y; ow[2] = a.z; ow[3] = a.w;
-            dw[0] = c.x; dw[1] = c.y; dw[2] = c.z; dw[3] = c.w;
+        } else if constexpr (NW % 4 != 0) {  // 8 or 24 bytes per lane: 8-byte aligned
+#pragma unroll
+            for (int w = 0; w < NW; w += 2) {
+                const uint2 a = reinterpret_cast<const uint2*>(o16)[w / 2];
+                const uint2 c = reinterpret_cast<const uint2*>(d16)[w / 2];
+                ow[w] = a.x; ow[w + 1] = a.y; dw[w] = c.x; dw[w + 1] = c.y;
+            }
+        } else {  // 16 or 32 bytes per lane
+#pragma unroll
+            for (int w = 0; w < NW; w += 4) {
+                const uint4 a = reinterpret_cast<const uint4*>(o16)[w / 4];
+                const uint4 c = reinterpret_cast<const uint4*>(d16)[w / 4];
+                ow[w] = a.x; ow[w + 1] = a.y; ow[w + 2] = a.z; ow[w + 3] = a.w;
+                dw[w] = c.x; dw[w + 1] = c.y; dw[w + 2] = c.z; dw[w + 3] = c.w;
+            }
         }
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
@@ -186,6 +194,13 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p)
         for (int c = 0; c < 3; ++c) {
             const float2 a = reinterpret_cast<const float2*>(src)[c];
             reinterpret_cast<uint32_t*>(dst)[c] = pack2<BF16>(a.x * p.scale, a.y * p.scale);
+        }
+    } else if constexpr (D > 256) {  // 12 or 16 values per lane: 16-byte loads, 8-byte stores
+#pragma unroll
+        for (int c = 0; c < D / 128; ++c) {
+            const float4 a = reinterpret_cast<const float4*>(src)[c];
+            reinterpret_cast<uint2*>(dst)[c] =
+                make_uint2(pack2<BF16>(a.x * p.scale, a.y * p.scale), pack2<BF16>(a.z * p.scale, a.w * p.scale));
         }
     } else if constexpr (D == 128) {
         const float4 a = *reinterpret_cast<const float4*>(src);

@@ -1,5 +1,5 @@
 // fa_bwd_wide.cuh -- dK / dV / dQ-partials kernel of the attention backward for head_dim
-// 192 and 256.
+// 192, 256, 384 and 512.
 //
 // Same arithmetic as the head_dim 128 kernel in fa_bwd.cuh (P recomputed from LSE,
 // dS = P (dP - D), dV = P^T dO, dK = scale dS^T Q, dQ partials reduced in fp32), with
@@ -23,6 +23,14 @@
 // dim 192, and the second head-dim half of dV^T, dK^T and dQ^T has 64 live lanes (the
 // other 64 are zero and never read).
 //
+// head_dim 384 and 512 ("[RFC] FA4 -- head_dim=256 & head_dim=512", Phase 4): a unit
+// also carries a window of OW = D / 2 output head dims (192 or 256), and computes dV,
+// dK and dQ for those dims only; the score contractions S = Q K^T and dP = dO V^T
+// still run over all D dims, in two phases through the same tiles: first the other
+// window's dims of Q, K, dO and V, then the unit's own, which stay in shared memory
+// for the transposed products.  So every key block is visited by two units, each
+// recomputing S and dP (2 x 2 of the 5 GEMMs), and K and V are loaded per phase.
+//
 // TMEM: S [0,64) | dP [64,128) | dQ^T half [128,256) | dV^T halves [256,384) | dK^T [384,512)
 #pragma once
 
@@ -32,9 +40,12 @@ namespace fa {
 
 template <int DIM, bool BF16>
 struct BwdWideCfg {
-    static_assert(DIM == 192 || DIM == 256, "head_dim");
+    static_assert(DIM == 192 || DIM == 256 || DIM == 384 || DIM == 512, "head_dim");
     static constexpr int D = DIM;
-    static constexpr int NB = D / 64;  // 64-dim blocks loaded per operand tile
+    static constexpr int OW = D > 256 ? D / 2 : D;  // output head dims per unit (window)
+    static constexpr int NWIN = D / OW;             // windows per key block
+    static constexpr int PH = NWIN;                 // contraction phases per step
+    static constexpr int NB = OW / 64;  // 64-dim blocks loaded per operand tile
     static constexpr int BN = 64;   // keys per unit
     static constexpr int BM = 128;  // query rows per step
     // warps 0-7: compute (two warpgroups, 32 keys each), 8-11: dQ, 12: MMA, 13: TMA,
@@ -43,7 +54,7 @@ struct BwdWideCfg {
     static constexpr int DQ_WARP = 8, MMA_WARP = 12, LOAD_WARP = 13;
     // registers per thread: launched at 128; the MMA/TMA warpgroup gives 8 of them to
     // the dQ warpgroup, which then holds a whole 128-column dQ^T row in registers
-    static constexpr uint32_t REG_LAUNCH = 128, REG_DQ = D == 256 ? 136 : 144, REG_CTRL = D == 256 ? 120 : 112;
+    static constexpr uint32_t REG_LAUNCH = 128, REG_DQ = OW == 256 ? 136 : 144, REG_CTRL = OW == 256 ? 120 : 112;
     static_assert(8 * 32 * REG_LAUNCH + 4 * 32 * REG_DQ + 4 * 32 * REG_CTRL <= THREADS * REG_LAUNCH,
                   "register split exceeds the launch budget");
     // lane 0 of the MMA warp issues alone (the converged, elected-lane form measured
@@ -63,7 +74,7 @@ struct BwdWideCfg {
     static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1, B_Q_FULL = 2, B_Q_EMPTY = 3, B_DO_FULL = 4,
                          B_DO_EMPTY = 5, B_S_FULL = 6, B_DP_FULL = 7, B_P_FULL = 8, B_P_EMPTY = 9,
                          B_DS_FULL = 10, B_DS_EMPTY = 11, B_DQ_FULL = 12, B_DQ_EMPTY = 13,
-                         B_DKV_FINAL = 14, B_DRAIN = 15, NBAR = 16;
+                         B_DKV_FINAL = 14, B_DRAIN = 15, B_ROWS_FULL = 16, B_ROWS_EMPTY = 17, NBAR = 18;
     static constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
     static constexpr uint32_t SMEM_BYTES = OFF_CTL + sizeof(CtaCtl);
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -77,12 +88,15 @@ enum : uint32_t {
     W_B256_KV_FULL = 0x301, W_B256_KV_EMPTY, W_B256_Q_FULL, W_B256_Q_EMPTY, W_B256_DO_FULL,
     W_B256_DO_EMPTY, W_B256_S_FULL, W_B256_DP_FULL, W_B256_P_FULL, W_B256_P_EMPTY,
     W_B256_DS_FULL, W_B256_DS_EMPTY, W_B256_DQ_FULL, W_B256_DQ_EMPTY, W_B256_DKV_FINAL,
-    W_B256_DRAIN, W_B256_SMEM_ALIGN
+    W_B256_DRAIN, W_B256_SMEM_ALIGN, W_B256_ROWS_FULL, W_B256_ROWS_EMPTY
 };
 
-// num_n counts 64-key blocks here
-__device__ __forceinline__ BwdUnit bwd_wide_decode(const BwdParams& p, int t)
+// num_n counts 64-key blocks here; the NWIN windows of one key block are adjacent
+template <int NWIN>
+__device__ __forceinline__ BwdUnit bwd_wide_decode(const BwdParams& p, int t, int& win)
 {
+    win = t % NWIN;
+    t /= NWIN;
     const int BH = p.B * p.Hkv;
     const int per_chunk = p.chunk_heads * p.num_n;
     const int c = t / per_chunk;
@@ -144,17 +158,20 @@ __device__ void bwd_wide_compute(const BwdParams& p, uint32_t tmem, uint32_t bas
     const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
     uint32_t it = 0, unit_it = 0;
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
-        const BwdUnit u = bwd_wide_decode(p, ui);
+        int win;
+        const BwdUnit u = bwd_wide_decode<C::NWIN>(p, ui, win);
         if (!u.keys) continue;  // past the end of its sequence's keys
-        // dV^T / dK^T element of head-dim column (hf * 128 + t) for key `key` of the unit
+        // dV^T / dK^T element of head-dim column (hf * 128 + t) of the unit's window for
+        // key `key` of the unit
         auto grad_off = [&](int key, int hf) {
-            return ((static_cast<size_t>(u.tb) * p.Sk_alloc + u.k_base + key) * p.Hkv + u.hkv) * C::D + hf * 128 + t;
+            return ((static_cast<size_t>(u.tb) * p.Sk_alloc + u.k_base + key) * p.Hkv + u.hkv) * C::D +
+                   win * C::OW + hf * 128 + t;
         };
         if (u.T == 0) {  // keys that no query of the sequence sees: zero gradients
             T* dst = static_cast<T*>(half == 0 ? p.dv : p.dk);
             for (int key = u.n * 64; key < min(u.n * 64 + 64, u.Sk); ++key)
                 for (int hf = 0; hf < 2; ++hf)
-                    if (D == 256 || hf * 128 + t < D) dst[grad_off(key, hf)] = static_cast<T>(0.0f);
+                    if (hf * 128 + t < C::OW) dst[grad_off(key, hf)] = static_cast<T>(0.0f);
             continue;
         }
         for (int s = 0; s < u.T; ++s, ++it) {
@@ -167,10 +184,12 @@ __device__ void bwd_wide_compute(const BwdParams& p, uint32_t tmem, uint32_t bas
             const int klim = u.Sk - 1 - u.n * 64;
             const int lim = p.causal ? min(i + (u.Sk - u.Sq) - u.n * 64, klim) : klim;
             const bool masked = (p.causal && (u.n * 64 + 63 > m * 128 + u.Sk - u.Sq)) || (u.n * 64 + 64 > u.Sk);
-            if (!warp_wait<true>(bar(C::B_Q_FULL), it & 1u, ctl, W_B256_Q_FULL)) return;
+            if (!warp_wait<true>(bar(C::B_ROWS_FULL), it & 1u, ctl, W_B256_ROWS_FULL)) return;
             float l2, dval;
-            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l2) : "r"(base + C::OFF_ROWS + t * 4u));
-            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dval) : "r"(base + C::OFF_ROWS + 512u + t * 4u));
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l2) : "r"(base + C::OFF_ROWS + t * 4u) : "memory");
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dval) : "r"(base + C::OFF_ROWS + 512u + t * 4u) : "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_ROWS_EMPTY));
             const uint64_t negl2 = f2pack(-l2, -l2);
             if (!warp_wait<true>(bar(C::B_S_FULL), it & 1u, ctl, W_B256_S_FULL)) return;
             tc_fence_after();
@@ -230,8 +249,8 @@ __device__ void bwd_wide_compute(const BwdParams& p, uint32_t tmem, uint32_t bas
             T* dst = static_cast<T*>(which == 0 ? p.dv : p.dk);
 #pragma unroll 1
             for (int hf = 0; hf < 2; ++hf) {
-                if constexpr (D < 256)
-                    if (hf * 128 + t >= D) break;  // a zero lane of the padded half
+                if constexpr (C::OW < 256)
+                    if (hf * 128 + t >= C::OW) break;  // a zero lane of the padded half
                 const uint32_t col = (which == 0 ? C::T_DV : C::T_DK) + hf * 64;
                 uint32_t r[32];
 #pragma unroll 1
@@ -260,7 +279,8 @@ __device__ void bwd_wide_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t b
     auto bar = [&](int i) { return bars + 8u * i; };
     uint32_t k = 0;  // dQ halves drained so far
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
-        const BwdUnit u = bwd_wide_decode(p, ui);
+        int win;
+        const BwdUnit u = bwd_wide_decode<C::NWIN>(p, ui, win);
         for (int s = 0; s < u.T; ++s) {
             int h, m;
             bwd_step(p, u, s, h, m);
@@ -268,8 +288,8 @@ __device__ void bwd_wide_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t b
 #pragma unroll 1
             for (int dh = 0; dh < 2; ++dh, ++k) {
                 if (!warp_wait<true>(bar(C::B_DQ_FULL), k & 1u, ctl, W_B256_DQ_FULL)) return;
-                if constexpr (D < 256) {
-                    if (dh * 128 + wq * 32 >= D) {  // zero lanes of the padded half
+                if constexpr (C::OW < 256) {
+                    if (dh * 128 + wq * 32 >= C::OW) {  // zero lanes of the padded half
                         if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
                         continue;
                     }
@@ -280,7 +300,7 @@ __device__ void bwd_wide_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t b
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
-                float* dst = blk + dh * 128;
+                float* dst = blk + win * C::OW + dh * 128;
                 red_rows<C::D * 4>(dst, r, std::make_index_sequence<128>{});
             }
         }
@@ -304,12 +324,12 @@ __device__ void bwd_wide_mma(const BwdParams& p, uint32_t tmem, uint32_t base, u
     const uint64_t mP = sdesc_sw128(sP, C::Q_BLK, 1024), mDS = sdesc_sw128(sDS, C::Q_BLK, 1024);
     const uint64_t kDS = sdesc_sw128(sDS, 16, 1024), mK = sdesc_sw128(sK, C::KV_BLK, 1024);
     // S (or dP) = X Y^T over d: X a [128][d] tile, Y a [64][d] tile
-    auto mma_qk = [&](uint32_t d_t, uint64_t x, uint64_t y) {
+    auto mma_qk = [&](uint32_t d_t, uint64_t x, uint64_t y, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < C::OW / 16; ++kk) {
             const uint32_t xo = ((kk >> 2) * C::Q_BLK + (kk & 3) * 32u) >> 4;
             const uint32_t yo = ((kk >> 2) * C::KV_BLK + (kk & 3) * 32u) >> 4;
-            I::ss(tmem + d_t, x + xo, y + yo, C::IDESC_S, kk > 0);
+            I::ss(tmem + d_t, x + xo, y + yo, C::IDESC_S, (acc || kk > 0) ? 1u : 0u);
         }
     };
     // acc^T[half] (+)= X^T Z: X a [128 query][d] tile read MN-major (head-dim half
@@ -334,18 +354,20 @@ __device__ void bwd_wide_mma(const BwdParams& p, uint32_t tmem, uint32_t base, u
         if (dq_issued == 0) return true;
         return I::wait(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_B256_DQ_EMPTY);
     };
+    if constexpr (C::PH == 1) {
     for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
-        const BwdUnit u = bwd_wide_decode(p, ui);
+        int win;
+        const BwdUnit u = bwd_wide_decode<C::NWIN>(p, ui, win);
         if (u.T == 0) continue;
         if (!I::wait(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_B256_KV_FULL)) return;
         tc_fence_after();
         if (!I::wait(bar(C::B_Q_FULL), it & 1u, ctl, W_B256_Q_FULL)) return;
         tc_fence_after();
-        mma_qk(C::T_S, kQ, kK);
+        mma_qk(C::T_S, kQ, kK, false);
         I::commit(bar(C::B_S_FULL));
         if (!I::wait(bar(C::B_DO_FULL), it & 1u, ctl, W_B256_DO_FULL)) return;
         tc_fence_after();
-        mma_qk(C::T_DP, kDO, kV);
+        mma_qk(C::T_DP, kDO, kV, false);
         I::commit(bar(C::B_DP_FULL));
         for (int s = 0; s < u.T; ++s, ++it) {
             if (!I::wait(bar(C::B_P_FULL), it & 1u, ctl, W_B256_P_FULL)) return;
@@ -365,11 +387,11 @@ __device__ void bwd_wide_mma(const BwdParams& p, uint32_t tmem, uint32_t base, u
             if (s + 1 < u.T) {
                 if (!I::wait(bar(C::B_Q_FULL), (it + 1) & 1u, ctl, W_B256_Q_FULL)) return;
                 tc_fence_after();
-                mma_qk(C::T_S, kQ, kK);
+                mma_qk(C::T_S, kQ, kK, false);
                 I::commit(bar(C::B_S_FULL));
                 if (!I::wait(bar(C::B_DO_FULL), (it + 1) & 1u, ctl, W_B256_DO_FULL)) return;
                 tc_fence_after();
-                mma_qk(C::T_DP, kDO, kV);
+                mma_qk(C::T_DP, kDO, kV, false);
                 I::commit(bar(C::B_DP_FULL));
             }
             if (!wait_dq_free()) return;
@@ -383,6 +405,66 @@ __device__ void bwd_wide_mma(const BwdParams& p, uint32_t tmem, uint32_t base, u
         I::commit(bar(C::B_DKV_FINAL));
         ++unit_it;
     }
+    } else {
+    // Two contraction phases per step: S and dP over the other window's dims, then over
+    // the unit's own (whose Q, dO and K tiles the transposed products read).  K / V,
+    // Q and dO each complete their FULL barrier once per phase.
+    uint32_t kv_it = 0, q_it = 0, do_it = 0;
+    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+        int win;
+        const BwdUnit u = bwd_wide_decode<C::NWIN>(p, ui, win);
+        if (u.T == 0) continue;
+        for (int s = 0; s < u.T; ++s, ++it) {
+            // phase A: the other window's dims
+            if (!I::wait(bar(C::B_KV_FULL), kv_it & 1u, ctl, W_B256_KV_FULL)) return;
+            if (!I::wait(bar(C::B_Q_FULL), q_it & 1u, ctl, W_B256_Q_FULL)) return;
+            tc_fence_after();
+            mma_qk(C::T_S, kQ, kK, false);
+            I::commit(bar(C::B_Q_EMPTY));
+            ++q_it;
+            if (!I::wait(bar(C::B_DO_FULL), do_it & 1u, ctl, W_B256_DO_FULL)) return;
+            tc_fence_after();
+            mma_qk(C::T_DP, kDO, kV, false);
+            I::commit(bar(C::B_DO_EMPTY));
+            ++do_it;
+            I::commit(bar(C::B_KV_EMPTY));
+            ++kv_it;
+            // phase B: the unit's own window
+            if (!I::wait(bar(C::B_KV_FULL), kv_it & 1u, ctl, W_B256_KV_FULL)) return;
+            if (!I::wait(bar(C::B_Q_FULL), q_it & 1u, ctl, W_B256_Q_FULL)) return;
+            tc_fence_after();
+            mma_qk(C::T_S, kQ, kK, true);
+            I::commit(bar(C::B_S_FULL));
+            if (!I::wait(bar(C::B_DO_FULL), do_it & 1u, ctl, W_B256_DO_FULL)) return;
+            tc_fence_after();
+            mma_qk(C::T_DP, kDO, kV, true);
+            I::commit(bar(C::B_DP_FULL));
+            if (!I::wait(bar(C::B_P_FULL), it & 1u, ctl, W_B256_P_FULL)) return;
+            tc_fence_after();
+            mma_t(C::T_DV, mDO, mP, s > 0);
+            I::commit(bar(C::B_P_EMPTY));
+            I::commit(bar(C::B_DO_EMPTY));
+            ++do_it;
+            if (!I::wait(bar(C::B_DS_FULL), it & 1u, ctl, W_B256_DS_FULL)) return;
+            tc_fence_after();
+            mma_t(C::T_DK, mQ, mDS, s > 0);
+            I::commit(bar(C::B_Q_EMPTY));
+            ++q_it;
+            for (int dh = 0; dh < 2; ++dh) {
+                if (!wait_dq_free()) return;
+                tc_fence_after();
+                mma_dq(dh);
+                I::commit(bar(C::B_DQ_FULL));
+                ++dq_issued;
+            }
+            I::commit(bar(C::B_DS_EMPTY));
+            I::commit(bar(C::B_KV_EMPTY));
+            ++kv_it;
+        }
+        I::commit(bar(C::B_DKV_FINAL));
+        ++unit_it;
+    }
+    }
 }
 
 // ---- TMA producer --------------------------------------------------------------------
@@ -392,54 +474,76 @@ struct BwdWideLoad {
     const CUtensorMap *tmQ, *tmK, *tmV, *tmDO;  // K, V maps have 64-row boxes
     uint32_t base, bars;
     CtaCtl* ctl;
-    int kv_round = -1, q_round = -1, do_round = -1;
+    // loads issued so far per barrier (the last one's FULL phase is drained at exit)
+    uint32_t kv_n = 0, q_n = 0, do_n = 0, rows_n = 0;
 
     __device__ uint32_t bar(int i) const { return bars + 8u * i; }
+    // K and V of the unit's 64 keys, head dims col0 .. col0 + OW - 1
+    __device__ bool load_kv(const BwdUnit& u, int col0)
+    {
+        if (!wait_bar_inl(bar(C::B_KV_EMPTY), (kv_n & 1u) ^ 1u, ctl, W_B256_KV_EMPTY)) return false;
+        mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::KV_LOAD);
+        for (int blk = 0; blk < C::NB; ++blk) {
+            tma_load_4d(base + C::OFF_K + blk * C::KV_BLK, tmK, bar(C::B_KV_FULL), col0 + blk * 64, u.hkv,
+                        u.k_base + u.n * 64, u.tb);
+            tma_load_4d(base + C::OFF_V + blk * C::KV_BLK, tmV, bar(C::B_KV_FULL), col0 + blk * 64, u.hkv,
+                        u.k_base + u.n * 64, u.tb);
+        }
+        ++kv_n;
+        return true;
+    }
+    // the 128-row Q (or dO) tile of query head h, block m, head dims col0 .. col0 + OW - 1
+    __device__ bool load_q(const CUtensorMap* tm, int full, int empty, uint32_t& n, uint32_t where,
+                           const BwdUnit& u, int h, int m, int col0)
+    {
+        if (!wait_bar_inl(bar(empty), (n & 1u) ^ 1u, ctl, where)) return false;
+        mbar_arrive_expect_tx(bar(full), C::Q_LOAD);
+        const uint32_t dst = base + (full == C::B_Q_FULL ? C::OFF_Q : C::OFF_DO);
+        for (int blk = 0; blk < C::NB; ++blk)
+            tma_load_4d(dst + blk * C::Q_BLK, tm, bar(full), col0 + blk * 64, h, u.q_base + m * 128, u.tb);
+        ++n;
+        return true;
+    }
+    // LSE*log2(e) and D of the 128 rows of query head h, block m
+    __device__ bool load_rows(const BwdParams& p, const BwdUnit& u, int h, int m)
+    {
+        if (!wait_bar_inl(bar(C::B_ROWS_EMPTY), (rows_n & 1u) ^ 1u, ctl, W_B256_ROWS_EMPTY)) return false;
+        mbar_arrive_expect_tx(bar(C::B_ROWS_FULL), C::ROWS_BYTES);
+        const size_t rb = (static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + static_cast<size_t>(m) * 128;
+        bulk_load(base + C::OFF_ROWS, p.L2 + rb, 512, bar(C::B_ROWS_FULL));
+        bulk_load(base + C::OFF_ROWS + 512, p.Dv + rb, 512, bar(C::B_ROWS_FULL));
+        ++rows_n;
+        return true;
+    }
     __device__ void run(const BwdParams& p)
     {
-        uint32_t it = 0, unit_it = 0;
         for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
-            const BwdUnit u = bwd_wide_decode(p, ui);
+            int win;
+            const BwdUnit u = bwd_wide_decode<C::NWIN>(p, ui, win);
             if (u.T == 0) continue;
-            if (!wait_bar_inl(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_B256_KV_EMPTY)) return;
-            mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::KV_LOAD);
-            for (int blk = 0; blk < C::NB; ++blk) {
-                tma_load_4d(base + C::OFF_K + blk * C::KV_BLK, tmK, bar(C::B_KV_FULL), blk * 64, u.hkv,
-                            u.k_base + u.n * 64, u.tb);
-                tma_load_4d(base + C::OFF_V + blk * C::KV_BLK, tmV, bar(C::B_KV_FULL), blk * 64, u.hkv,
-                            u.k_base + u.n * 64, u.tb);
-            }
-            kv_round = static_cast<int>(unit_it);
-            ++unit_it;
-            for (int s = 0; s < u.T; ++s, ++it) {
+            if constexpr (C::PH == 1)
+                if (!load_kv(u, 0)) return;
+            for (int s = 0; s < u.T; ++s) {
                 int h, m;
                 bwd_step(p, u, s, h, m);
-                const uint32_t ph = (it & 1u) ^ 1u;
-                if (!wait_bar_inl(bar(C::B_Q_EMPTY), ph, ctl, W_B256_Q_EMPTY)) return;
-                mbar_arrive_expect_tx(bar(C::B_Q_FULL), C::Q_LOAD + C::ROWS_BYTES);
-                for (int blk = 0; blk < C::NB; ++blk)
-                    tma_load_4d(base + C::OFF_Q + blk * C::Q_BLK, tmQ, bar(C::B_Q_FULL), blk * 64, h,
-                                u.q_base + m * 128, u.tb);
-                {
-                    const size_t rb = (static_cast<size_t>(u.b) * p.Hq + h) * p.Sq_pad + static_cast<size_t>(m) * 128;
-                    bulk_load(base + C::OFF_ROWS, p.L2 + rb, 512, bar(C::B_Q_FULL));
-                    bulk_load(base + C::OFF_ROWS + 512, p.Dv + rb, 512, bar(C::B_Q_FULL));
+                // in the MMA issuer's order: per phase K / V (two phases only), Q, then
+                // the rows once per step, then dO
+                for (int ph = 0; ph < C::PH; ++ph) {
+                    const int col0 = (C::PH == 1 ? 0 : (ph == 0 ? 1 - win : win)) * C::OW;
+                    if (C::PH > 1 && !load_kv(u, col0)) return;
+                    if (!load_q(tmQ, C::B_Q_FULL, C::B_Q_EMPTY, q_n, W_B256_Q_EMPTY, u, h, m, col0)) return;
+                    if (ph == C::PH - 1 && !load_rows(p, u, h, m)) return;
+                    if (!load_q(tmDO, C::B_DO_FULL, C::B_DO_EMPTY, do_n, W_B256_DO_EMPTY, u, h, m, col0)) return;
                 }
-                q_round = static_cast<int>(it);
-                if (!wait_bar_inl(bar(C::B_DO_EMPTY), ph, ctl, W_B256_DO_EMPTY)) return;
-                mbar_arrive_expect_tx(bar(C::B_DO_FULL), C::Q_LOAD);
-                for (int blk = 0; blk < C::NB; ++blk)
-                    tma_load_4d(base + C::OFF_DO + blk * C::Q_BLK, tmDO, bar(C::B_DO_FULL), blk * 64, h,
-                                u.q_base + m * 128, u.tb);
-                do_round = static_cast<int>(it);
             }
         }
     }
     __device__ void drain()
     {
-        if (kv_round >= 0) drain_wait_inl(bar(C::B_KV_FULL), static_cast<uint32_t>(kv_round) & 1u, W_B256_DRAIN);
-        if (q_round >= 0) drain_wait_inl(bar(C::B_Q_FULL), static_cast<uint32_t>(q_round) & 1u, W_B256_DRAIN);
-        if (do_round >= 0) drain_wait_inl(bar(C::B_DO_FULL), static_cast<uint32_t>(do_round) & 1u, W_B256_DRAIN);
+        if (kv_n) drain_wait_inl(bar(C::B_KV_FULL), (kv_n - 1u) & 1u, W_B256_DRAIN);
+        if (q_n) drain_wait_inl(bar(C::B_Q_FULL), (q_n - 1u) & 1u, W_B256_DRAIN);
+        if (do_n) drain_wait_inl(bar(C::B_DO_FULL), (do_n - 1u) & 1u, W_B256_DRAIN);
+        if (rows_n) drain_wait_inl(bar(C::B_ROWS_FULL), (rows_n - 1u) & 1u, W_B256_DRAIN);
     }
 };
 
@@ -468,6 +572,7 @@ __global__ void __launch_bounds__(BwdWideCfg<D, BF16>::THREADS, 1)
         mbar_init(bar(C::B_P_FULL), 8);
         mbar_init(bar(C::B_DS_FULL), 8);
         mbar_init(bar(C::B_DQ_EMPTY), 4);
+        mbar_init(bar(C::B_ROWS_EMPTY), 8);  // one arrive per compute warp
         ctl->abort = 0u;
         fence_mbar_init();
     }

@@ -24,10 +24,9 @@
  *   - causal != 0 applies a lower-triangular mask aligned to the bottom-right
  *     corner: key j is visible to query i iff j <= i + (Sk - Sq).
  *   - head_dim d must be 128, 192, 256, 384 or 512 (192, 384, 512: "[RFC] FA4 --
- *     head_dim=256 & head_dim=512", Phase 4, symmetric head dims; the backward
- *     entry points take d up to 256 and return FA_ERR_UNSUPPORTED above); dtype
- *     must be FA_BF16 or FA_FP16 and is the same for every 16-bit tensor of a call.
- *     Every pointer must be 16-byte aligned.
+ *     head_dim=256 & head_dim=512", Phase 4, symmetric head dims); dtype must be
+ *     FA_BF16 or FA_FP16 and is the same for every 16-bit tensor of a call.  Every
+ *     pointer must be 16-byte aligned.
  *   - Ownership: the caller owns every buffer.  The library allocates no device
  *     memory per call; scratch for the backward is the caller's workspace.
  *     Work is enqueued on `stream` and runs asynchronously; nothing synchronises.
