@@ -18,6 +18,7 @@ library's CUDA kernels.  The functions carry the C names:
     fa_clear_device_status()
     fa_set_unit_schedule(mode)        # FA_SCHED_STATIC (0, default) or FA_SCHED_CLC (1)
     fa_set_exp2_emulation(pairs_of_4) # forward exp2 split: -1 default, 0..3 of 4 on the FMA pipe
+    fa_set_wait_timeout_ms(ms)        # limit of a kernel's pipeline waits (default 1000)
     fa_debug_inject(mode)
     fa_debug_exp2(x, mode=0) -> y
 
@@ -35,7 +36,7 @@ from . import _lib
 
 __all__ = [
     "FAError", "fa_fwd", "fa_fwd_splitkv", "fa_fwd_varlen", "fa_bwd", "fa_bwd_varlen", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
-    "fa_last_device_status", "fa_clear_device_status", "fa_set_unit_schedule", "fa_set_exp2_emulation", "fa_debug_inject", "fa_debug_exp2",
+    "fa_last_device_status", "fa_clear_device_status", "fa_set_unit_schedule", "fa_set_exp2_emulation", "fa_set_wait_timeout_ms", "fa_debug_inject", "fa_debug_exp2",
     "FA_SCHED_STATIC", "FA_SCHED_CLC",
 ]
 
@@ -339,6 +340,13 @@ def fa_set_exp2_emulation(pairs_of_4: int):
     score tile use the FMA-pipe cubic instead of the special-function unit (0..3), or
     -1 for the library's per-head-dim default.  Process-wide."""
     _raise(_lib.load().fa_set_exp2_emulation(int(pairs_of_4)), "fa_set_exp2_emulation")
+
+
+def fa_set_wait_timeout_ms(ms: int):
+    """Limit (ms, 1..600000; 1000 initially) after which a kernel's pipeline wait gives
+    up and reports FA_ERR_DEVICE_TIMEOUT.  Wall-clock time on the device: raise it on
+    GPUs time-sliced between processes.  Process-wide."""
+    _raise(_lib.load().fa_set_wait_timeout_ms(int(ms)), "fa_set_wait_timeout_ms")
 
 
 def fa_debug_inject(mode: int):

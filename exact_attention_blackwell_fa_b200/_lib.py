@@ -38,6 +38,7 @@ SIGNATURES = {
     "fa_debug_inject": (_ci, [_ci]),
     "fa_set_unit_schedule": (_ci, [_ci]),
     "fa_set_exp2_emulation": (_ci, [_ci]),
+    "fa_set_wait_timeout_ms": (_ci, [_ci]),
     "fa_debug_exp2": (_ci, [_vp, _vp, _ci, _ci, _vp]),
 }
 

@@ -132,6 +132,7 @@ int g_inject = 0;
 std::mutex g_inject_mu;
 std::atomic<int> g_schedule{FA_SCHED_STATIC};
 std::atomic<int> g_exp2_emu{-1};  // -1: the per-head-dim default
+std::atomic<uint64_t> g_wait_ns{fa::kWaitTimeoutNs};  // limit of a kernel's pipeline waits
 
 int take_inject()
 {
@@ -329,6 +330,7 @@ static fa_status fwd_common(const void* q, const void* k, const void* v, void* o
     p.causal = causal ? 1 : 0;
     p.inject = take_inject();
     p.sl2 = scale * 1.4426950408889634f;
+    p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     st = launch_fwd_any(d, bf16, tq, tk, tv, p, di.sm_count, s);
     if (st != FA_OK || splits == 1) return st;
@@ -456,6 +458,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
     p.causal = causal ? 1 : 0;
     p.inject = take_inject();
     p.sl2 = scale * 1.4426950408889634f;
+    p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     return launch_fwd_any(d, bf16, tq, tk, tv, p, di.sm_count, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -532,6 +535,7 @@ static fa_status bwd_common(const void* q, const void* k, const void* v, const v
     p.causal = causal ? 1 : 0;
     p.scale = scale;
     p.sl2 = scale * 1.4426950408889634f;
+    p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (d == 512)
         return bf16 ? launch_bwd_wide<512, true>(tq, tk, tv, tdo, p, di.sm_count, s)
@@ -630,6 +634,13 @@ fa_status fa_set_exp2_emulation(int pairs_of_4)
 {
     if (pairs_of_4 < -1 || pairs_of_4 > 3) return FA_ERR_INVALID_ARG;
     g_exp2_emu.store(pairs_of_4, std::memory_order_relaxed);
+    return FA_OK;
+}
+
+fa_status fa_set_wait_timeout_ms(int ms)
+{
+    if (ms < 1 || ms > 600000) return FA_ERR_INVALID_ARG;
+    g_wait_ns.store(static_cast<uint64_t>(ms) * 1000000ull, std::memory_order_relaxed);
     return FA_OK;
 }
 

@@ -67,6 +67,7 @@ struct BwdParams {
     int chunk_heads;  // KV heads per L2 group in the unit order
     int causal;
     float scale, sl2;
+    uint64_t wait_ns;  // limit of a pipeline wait (see CtaCtl)
 };
 
 enum : uint32_t {
@@ -673,10 +674,13 @@ struct BwdLoad {
     }
     __device__ void drain()
     {
-        if (kv_round >= 0) drain_wait_inl(bar(C::B_KV_FULL), static_cast<uint32_t>(kv_round) & 1u, W_BWD_DRAIN);
+        const uint64_t lim = drain_limit(ctl);
+        if (kv_round >= 0) drain_wait_inl(bar(C::B_KV_FULL), static_cast<uint32_t>(kv_round) & 1u, W_BWD_DRAIN, lim);
         for (int st = 0; st < 2; ++st) {
-            if (q_round[st] >= 0) drain_wait_inl(bar(C::B_Q_FULL + st), static_cast<uint32_t>(q_round[st]) & 1u, W_BWD_DRAIN);
-            if (do_round[st] >= 0) drain_wait_inl(bar(C::B_DO_FULL + st), static_cast<uint32_t>(do_round[st]) & 1u, W_BWD_DRAIN);
+            if (q_round[st] >= 0)
+                drain_wait_inl(bar(C::B_Q_FULL + st), static_cast<uint32_t>(q_round[st]) & 1u, W_BWD_DRAIN, lim);
+            if (do_round[st] >= 0)
+                drain_wait_inl(bar(C::B_DO_FULL + st), static_cast<uint32_t>(do_round[st]) & 1u, W_BWD_DRAIN, lim);
         }
     }
 };
@@ -720,6 +724,7 @@ __global__ void __launch_bounds__(BwdCfg<BF16>::THREADS, 1)
         mbar_init(bar(C::B_DKV_FINAL), 1);
         mbar_init(bar(C::B_DRAIN), 1);
         ctl->abort = 0u;
+        ctl->wait_ns = p.wait_ns;
         fence_mbar_init();
     }
     if (warp == C::MMA_WARP) {
@@ -749,7 +754,7 @@ __global__ void __launch_bounds__(BwdCfg<BF16>::THREADS, 1)
             if (C::WARP_ISSUE || lane == 0) {
                 bwd_mma<BF16>(p, tmem, base, bars, ctl);
                 Issuer<C::WARP_ISSUE, true, true>::commit(bars + 8u * C::B_DRAIN);
-                if (lane == 0) drain_wait_inl(bars + 8u * C::B_DRAIN, 0u, W_BWD_DRAIN);
+                if (lane == 0) drain_wait_inl(bars + 8u * C::B_DRAIN, 0u, W_BWD_DRAIN, drain_limit(ctl));
             }
             __syncwarp();
         } else if (warp == C::LOAD_WARP) {

@@ -540,10 +540,11 @@ struct BwdWideLoad {
     }
     __device__ void drain()
     {
-        if (kv_n) drain_wait_inl(bar(C::B_KV_FULL), (kv_n - 1u) & 1u, W_B256_DRAIN);
-        if (q_n) drain_wait_inl(bar(C::B_Q_FULL), (q_n - 1u) & 1u, W_B256_DRAIN);
-        if (do_n) drain_wait_inl(bar(C::B_DO_FULL), (do_n - 1u) & 1u, W_B256_DRAIN);
-        if (rows_n) drain_wait_inl(bar(C::B_ROWS_FULL), (rows_n - 1u) & 1u, W_B256_DRAIN);
+        const uint64_t lim = drain_limit(ctl);
+        if (kv_n) drain_wait_inl(bar(C::B_KV_FULL), (kv_n - 1u) & 1u, W_B256_DRAIN, lim);
+        if (q_n) drain_wait_inl(bar(C::B_Q_FULL), (q_n - 1u) & 1u, W_B256_DRAIN, lim);
+        if (do_n) drain_wait_inl(bar(C::B_DO_FULL), (do_n - 1u) & 1u, W_B256_DRAIN, lim);
+        if (rows_n) drain_wait_inl(bar(C::B_ROWS_FULL), (rows_n - 1u) & 1u, W_B256_DRAIN, lim);
     }
 };
 
@@ -574,6 +575,7 @@ __global__ void __launch_bounds__(BwdWideCfg<D, BF16>::THREADS, 1)
         mbar_init(bar(C::B_DQ_EMPTY), 4);
         mbar_init(bar(C::B_ROWS_EMPTY), 8);  // one arrive per compute warp
         ctl->abort = 0u;
+        ctl->wait_ns = p.wait_ns;
         fence_mbar_init();
     }
     if (warp == C::MMA_WARP) {
@@ -617,7 +619,7 @@ __global__ void __launch_bounds__(BwdWideCfg<D, BF16>::THREADS, 1)
             if (C::WARP_ISSUE || lane == 0) {
                 bwd_wide_mma<D, BF16>(p, tmem, base, bars, ctl);
                 Issuer<C::WARP_ISSUE, true>::commit(bars + 8u * C::B_DRAIN);
-                if (lane == 0) drain_wait_inl(bars + 8u * C::B_DRAIN, 0u, W_B256_DRAIN);
+                if (lane == 0) drain_wait_inl(bars + 8u * C::B_DRAIN, 0u, W_B256_DRAIN, drain_limit(ctl));
             }
             __syncwarp();
         } else if (warp == C::LOAD_WARP) {

@@ -11,7 +11,12 @@
 
 namespace fa {
 
-// Every wait in the kernels gives up after this long and reports FA_ERR_DEVICE_TIMEOUT.
+// Every pipeline wait in the kernels gives up after CtaCtl::wait_ns (the launch's
+// setting, fa_set_wait_timeout_ms; this by default) and reports FA_ERR_DEVICE_TIMEOUT.
+// The limit is wall-clock time (%globaltimer), which keeps running while the GPU
+// serves another context, so a time slice longer than the limit reads as a timeout.
+// Drains -- waits for copies and MMAs already issued, which always complete -- allow
+// at least this much whatever the setting.
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;
 // Spinning waits (SPIN below) first poll without suspending (test_wait) for this many
 // probes, then fall back to the suspending, timed loop: a thread suspended in try_wait
@@ -27,8 +32,14 @@ __device__ uint32_t g_status[4];
 // Per-CTA control block in shared memory.
 struct CtaCtl {
     uint32_t tmem_base;
-    uint32_t abort;  // set when any wait of this CTA gave up; other waits then bail out
+    uint32_t abort;    // set when any wait of this CTA gave up; other waits then bail out
+    uint64_t wait_ns;  // limit of a pipeline wait, from the launch parameters
 };
+
+__device__ __forceinline__ uint64_t drain_limit(const CtaCtl* ctl)
+{
+    return ctl->wait_ns > kWaitTimeoutNs ? ctl->wait_ns : kWaitTimeoutNs;
+}
 
 __device__ __forceinline__ void record_timeout(uint32_t where)
 {
@@ -39,19 +50,22 @@ __device__ __forceinline__ void record_timeout(uint32_t where)
 }
 
 // Single-thread bounded wait.  Returns false (and raises the CTA abort flag) if the
-// phase did not complete within kWaitTimeoutNs, or if another wait already aborted.
+// phase did not complete within ctl->wait_ns, or if another wait already aborted.
 // The _inl forms are for kernels that change per-warpgroup register budgets
 // (setmaxnreg): their code may not call out-of-line functions.
 __device__ __forceinline__ bool wait_bar_inl(uint32_t bar, uint32_t parity, CtaCtl* ctl, uint32_t where)
 {
     if (mbar_try_wait(bar, parity)) return true;
     volatile uint32_t* abort = &ctl->abort;
+    // the limit is read from shared memory at each check rather than held in registers
+    // (code under a tight setmaxnreg budget inlines this loop)
+    volatile const uint64_t* limit = &ctl->wait_ns;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 31u) == 0u) {
             if (*abort) return false;
-            if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+            if (global_timer_ns() - t0 > *limit) {
                 *abort = 1u;
                 record_timeout(where);
                 return false;
@@ -67,11 +81,12 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, CtaCtl* ctl
 
 // Bounded wait that ignores the abort flag: used while draining in-flight copies or
 // MMAs before the CTA exits, which always complete on their own.
-__device__ __forceinline__ bool drain_wait_inl(uint32_t bar, uint32_t parity, uint32_t where)
+__device__ __forceinline__ bool drain_wait_inl(uint32_t bar, uint32_t parity, uint32_t where,
+                                               uint64_t limit = kWaitTimeoutNs)
 {
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        if (global_timer_ns() - t0 > limit) {
             record_timeout(where);
             return false;
         }
@@ -79,9 +94,9 @@ __device__ __forceinline__ bool drain_wait_inl(uint32_t bar, uint32_t parity, ui
     return true;
 }
 
-__device__ __noinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32_t where)
+__device__ __noinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32_t where, uint64_t limit)
 {
-    return drain_wait_inl(bar, parity, where);
+    return drain_wait_inl(bar, parity, where, limit);
 }
 
 // The timed waits, inlined (INL) or called.  Code that runs under a setmaxnreg budget
@@ -93,10 +108,11 @@ __device__ __forceinline__ bool wait_bar_t(uint32_t bar, uint32_t parity, CtaCtl
     else return wait_bar(bar, parity, ctl, where);
 }
 template <bool INL>
-__device__ __forceinline__ bool drain_wait_t(uint32_t bar, uint32_t parity, uint32_t where)
+__device__ __forceinline__ bool drain_wait_t(uint32_t bar, uint32_t parity, uint32_t where,
+                                             uint64_t limit = kWaitTimeoutNs)
 {
-    if constexpr (INL) return drain_wait_inl(bar, parity, where);
-    else return drain_wait(bar, parity, where);
+    if constexpr (INL) return drain_wait_inl(bar, parity, where, limit);
+    else return drain_wait(bar, parity, where, limit);
 }
 
 // Single-thread wait: one inline probe (SPIN: a bounded non-suspending poll), then the

@@ -86,6 +86,7 @@ struct FwdParams {
     // cancelling CTAs that have not started (cluster launch control), in unit order.
     // clc == 0: a persistent grid walks the units with a static stride.
     int clc;
+    uint64_t wait_ns;  // limit of a pipeline wait (see CtaCtl)
 };
 
 // wait-site codes reported through the device status word
@@ -871,10 +872,12 @@ struct FwdLoad {
     {
         for (int i = 0; i < C::NSTAGE; ++i)
             if (filled[i] >= 0)
-                drain_wait_t<C::INL>(bar(C::B_FULL + i), static_cast<uint32_t>(filled[i]) & 1u, W_FWD_DRAIN);
-        if (q_round >= 0) drain_wait_t<C::INL>(bar(C::B_Q_FULL), static_cast<uint32_t>(q_round) & 1u, W_FWD_DRAIN);
+                drain_wait_t<C::INL>(bar(C::B_FULL + i), static_cast<uint32_t>(filled[i]) & 1u, W_FWD_DRAIN,
+                                     drain_limit(ctl));
+        if (q_round >= 0)
+            drain_wait_t<C::INL>(bar(C::B_Q_FULL), static_cast<uint32_t>(q_round) & 1u, W_FWD_DRAIN, drain_limit(ctl));
         // an unanswered cancellation request still writes its response
-        if (clc_pending) drain_wait_t<C::INL>(bar(C::B_CLC), clc_it & 1u, W_FWD_DRAIN);
+        if (clc_pending) drain_wait_t<C::INL>(bar(C::B_CLC), clc_it & 1u, W_FWD_DRAIN, drain_limit(ctl));
     }
 };
 
@@ -923,6 +926,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
         }
         mbar_init(bar(C::B_CLC), 1);
         ctl->abort = 0u;
+        ctl->wait_ns = p.wait_ns;
         fence_mbar_init();
     }
     if (warp == C::CTRL_WARP) {
@@ -952,7 +956,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BF16>::THREADS, 1)
                 mma.run(p);
                 // all MMAs issued by this warp must finish before TMEM is released
                 M::commit(bars + 8u * C::B_DRAIN);
-                if (lane == 0) drain_wait_t<C::INL>(bars + 8u * C::B_DRAIN, 0u, W_FWD_DRAIN);
+                if (lane == 0) drain_wait_t<C::INL>(bars + 8u * C::B_DRAIN, 0u, W_FWD_DRAIN, drain_limit(ctl));
             }
             __syncwarp();
         } else if (warp == C::CTRL_WARP + 1) {

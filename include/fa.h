@@ -193,13 +193,27 @@ const char* fa_status_string(fa_status s);
 /*
  * Device-side status of the kernels run so far on this device: FA_OK, or
  * FA_ERR_DEVICE_TIMEOUT if some kernel gave up on a bounded wait (each wait in
- * the kernels gives up after about one second).  Synchronises `stream` to read
- * it.  `detail` (may be NULL) receives a code naming the wait that gave up.
+ * the kernels gives up after the limit of fa_set_wait_timeout_ms, one second by
+ * default).  Synchronises `stream` to read it.  `detail` (may be NULL) receives a
+ * code naming the wait that gave up.  After a timeout the outputs of the calls
+ * since the last clear are invalid; the context stays usable.
  */
 fa_status fa_last_device_status(fa_stream stream, uint32_t* detail);
 
 /* Resets the device-side status to FA_OK (enqueued on `stream`). */
 fa_status fa_clear_device_status(fa_stream stream);
+
+/*
+ * Limit, in milliseconds (1 .. 600000; 1000 initially), after which a kernel's wait
+ * for a pipeline stage gives up, drains what it has in flight, records
+ * FA_ERR_DEVICE_TIMEOUT and returns, instead of spinning forever on a stage that
+ * will not come.  The limit is measured in wall-clock time on the device, which
+ * keeps running while the GPU serves another process: on a time-sliced GPU a slice
+ * longer than the limit reads as a timeout, so raise it there.  Process-wide;
+ * applies to launches made after the call.  Out-of-range values return
+ * FA_ERR_INVALID_ARG.
+ */
+fa_status fa_set_wait_timeout_ms(int ms);
 
 /*
  * Order in which the forward's CTAs take their work units ("[RFC] FA4 --

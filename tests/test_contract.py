@@ -164,3 +164,11 @@ def test_wide_head_dims_reach_the_device_check(lib):
     for d in (384, 512):
         assert fwd_call(lib, d=d) in (FA_ERR_CUDA, FA_ERR_UNSUPPORTED)
         assert bwd_call(lib, d=d) in (FA_ERR_CUDA, FA_ERR_UNSUPPORTED)
+
+
+def test_wait_timeout_setting_validated(lib):
+    for ms in (1, 50, 1000, 600000):
+        assert lib.fa_set_wait_timeout_ms(ms) == FA_OK
+    for ms in (0, -5, 600001):
+        assert lib.fa_set_wait_timeout_ms(ms) == FA_ERR_INVALID_ARG
+    assert lib.fa_set_wait_timeout_ms(1000) == FA_OK

@@ -50,3 +50,36 @@ def test_withheld_tile_reports_timeout_then_recovers(oracle_mod, d):
     half_ulp = torch.ldexp(torch.ones_like(o_ref), (e - 8).to(torch.int32))
     assert (err - (1e-2 + half_ulp)).max().item() <= 0.0, err.max().item()
     assert err.mean().item() <= 1e-3
+
+
+def test_wait_limit_is_configurable(oracle_mod):
+    """fa_set_wait_timeout_ms shortens the limit: the withheld-tile launch gives up in
+    well under the default second; restoring the default leaves the next launch
+    correct."""
+    import exact_attention_blackwell_fa_b200 as fa
+
+    shape = Shape(1, 256, 256, 2, 2, 128)
+    q, k, v = make_inputs(shape, seed=4)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    fa.fa_fwd(qc, kc, vc)  # warm: first-launch set-up outside the timed part
+    torch.cuda.synchronize()
+    fa.fa_clear_device_status()
+    try:
+        fa.fa_set_wait_timeout_ms(100)
+        fa.fa_debug_inject(1)
+        t0 = time.time()
+        fa.fa_fwd(qc, kc, vc)
+        torch.cuda.synchronize()
+        elapsed = time.time() - t0
+    finally:
+        fa.fa_set_wait_timeout_ms(1000)
+    code, detail = fa.fa_last_device_status()
+    assert code == FA_ERR_DEVICE_TIMEOUT, (code, hex(detail))
+    assert elapsed < 0.9, elapsed
+    fa.fa_clear_device_status()
+    o, _ = fa.fa_fwd(qc, kc, vc)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status()[0] == 0
+    o_ref, _ = oracle_mod.fwd(q, k, v)
+    err = (o.cpu().double() - o_ref).abs()
+    assert err.max().item() <= 1e-2 + 2.0 ** -8 * o_ref.abs().max().item() and err.mean().item() <= 1e-3
