@@ -59,6 +59,8 @@ CASES = [
     (1, 64, 64, 2, 2, 128, True),
     (1, 40, 50, 4, 2, 192, True),   # the library's head dims 192 and 256
     (1, 24, 24, 2, 2, 256, False),
+    (1, 20, 28, 2, 1, 384, True),   # and 384, 512
+    (1, 18, 18, 2, 2, 512, False),
 ]
 
 
