@@ -16,7 +16,7 @@ library's CUDA kernels.  The functions carry the C names:
     fa_status_string(code) -> str
     fa_last_device_status() -> (code, detail)
     fa_clear_device_status()
-    fa_set_unit_schedule(mode)        # FA_SCHED_STATIC (0, default) or FA_SCHED_CLC (1)
+    fa_set_unit_schedule(mode)        # FA_SCHED_STATIC (0), FA_SCHED_CLC (1), FA_SCHED_AUTO (2, default)
     fa_set_exp2_emulation(pairs_of_4) # forward exp2 split: -1 default, 0..3 of 4 on the FMA pipe
     fa_set_wait_timeout_ms(ms)        # limit of a kernel's pipeline waits (default 1000)
     fa_debug_inject(mode)
@@ -37,10 +37,10 @@ from . import _lib
 __all__ = [
     "FAError", "fa_fwd", "fa_fwd_splitkv", "fa_fwd_varlen", "fa_bwd", "fa_bwd_varlen", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string",
     "fa_last_device_status", "fa_clear_device_status", "fa_set_unit_schedule", "fa_set_exp2_emulation", "fa_set_wait_timeout_ms", "fa_debug_inject", "fa_debug_exp2",
-    "FA_SCHED_STATIC", "FA_SCHED_CLC",
+    "FA_SCHED_STATIC", "FA_SCHED_CLC", "FA_SCHED_AUTO",
 ]
 
-FA_SCHED_STATIC, FA_SCHED_CLC = 0, 1
+FA_SCHED_STATIC, FA_SCHED_CLC, FA_SCHED_AUTO = 0, 1, 2
 
 
 class FAError(RuntimeError):
@@ -329,9 +329,10 @@ def fa_clear_device_status(stream=None):
 
 
 def fa_set_unit_schedule(mode: int):
-    """Forward unit order: FA_SCHED_STATIC (persistent grid, fixed stride; default) or
+    """Forward unit order: FA_SCHED_STATIC (persistent grid, fixed stride),
     FA_SCHED_CLC (one CTA per unit, running CTAs cancel pending ones to take their
-    units).  Process-wide."""
+    units) or FA_SCHED_AUTO (the default: CLC for causal launches over >= 4096 keys,
+    else STATIC).  Process-wide."""
     _raise(_lib.load().fa_set_unit_schedule(int(mode)), "fa_set_unit_schedule")
 
 

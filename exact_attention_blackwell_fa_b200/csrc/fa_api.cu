@@ -130,7 +130,7 @@ fa_status check_regs(K kernel, int launch_regs)
 
 int g_inject = 0;
 std::mutex g_inject_mu;
-std::atomic<int> g_schedule{FA_SCHED_STATIC};
+std::atomic<int> g_schedule{FA_SCHED_AUTO};
 std::atomic<int> g_exp2_emu{-1};  // -1: the per-head-dim default
 std::atomic<uint64_t> g_wait_ns{fa::kWaitTimeoutNs};  // limit of a kernel's pipeline waits
 
@@ -232,9 +232,11 @@ fa_status launch_fwd_emu(int emu, const CUtensorMap& tq, const CUtensorMap& tk, 
 fa_status launch_fwd_any(int d, bool bf16, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          fa::FwdParams p, int sm_count, cudaStream_t s)
 {
-    // dynamic unit order (cluster launch control) when selected and there are more
-    // units than SMs
-    p.clc = (g_schedule.load(std::memory_order_relaxed) == FA_SCHED_CLC && p.num_tiles > sm_count) ? 1 : 0;
+    // dynamic unit order (cluster launch control) when selected, or by default for
+    // causal launches over >= 4096 keys, and there are more units than SMs
+    const int mode = g_schedule.load(std::memory_order_relaxed);
+    const bool dynamic = mode == FA_SCHED_CLC || (mode == FA_SCHED_AUTO && p.causal && p.Sk >= 4096);
+    p.clc = (dynamic && p.num_tiles > sm_count) ? 1 : 0;
     int emu = g_exp2_emu.load(std::memory_order_relaxed);
     if (emu < 0) emu = exp2_emulation_default(d);
     switch (d) {
@@ -625,7 +627,7 @@ fa_status fa_debug_exp2(const float* x, float* y, int n, int mode, fa_stream str
 
 fa_status fa_set_unit_schedule(int mode)
 {
-    if (mode != FA_SCHED_STATIC && mode != FA_SCHED_CLC) return FA_ERR_INVALID_ARG;
+    if (mode != FA_SCHED_STATIC && mode != FA_SCHED_CLC && mode != FA_SCHED_AUTO) return FA_ERR_INVALID_ARG;
     g_schedule.store(mode, std::memory_order_relaxed);
     return FA_OK;
 }

@@ -321,7 +321,7 @@ __device__ void bwd_compute(const BwdParams& p, uint32_t tmem, uint32_t sDS, uin
     auto bar = [&](int i) { return bars + 8u * i; };
     const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
     uint32_t it = 0, unit_it = 0;
-    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+    for (int rnd = 0, ui = walk_unit(0); ui < p.num_units; ui = walk_unit(++rnd)) {
         const BwdUnit u = bwd_decode(p, ui);
         if (!u.keys) continue;  // past the end of its sequence's keys
         const int j = u.n * 128 + t;  // key row
@@ -496,7 +496,7 @@ __device__ void bwd_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t bars, 
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     auto bar = [&](int i) { return bars + 8u * i; };
     uint32_t it = 0;
-    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+    for (int rnd = 0, ui = walk_unit(0); ui < p.num_units; ui = walk_unit(++rnd)) {
         const BwdUnit u = bwd_decode(p, ui);
         for (int s = 0; s < u.T; ++s, ++it) {
             int h, m;
@@ -550,7 +550,7 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t tmem, uint32_t base, uint32
         if (dq_issued == 0) return true;
         return I::wait(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_BWD_DQ_EMPTY);
     };
-    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+    for (int rnd = 0, ui = walk_unit(0); ui < p.num_units; ui = walk_unit(++rnd)) {
         const BwdUnit u = bwd_decode(p, ui);
         if (u.T == 0) continue;
         if (!I::wait(bar(C::B_KV_FULL), unit_it & 1u, ctl, W_BWD_KV_FULL)) return;
@@ -640,7 +640,7 @@ struct BwdLoad {
     __device__ void run(const BwdParams& p)
     {
         uint32_t it = 0, unit_it = 0;
-        for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+        for (int rnd = 0, ui = walk_unit(0); ui < p.num_units; ui = walk_unit(++rnd)) {
             const BwdUnit u = bwd_decode(p, ui);
             if (u.T == 0) continue;
             if (!wait_bar_inl(bar(C::B_KV_EMPTY), (unit_it & 1u) ^ 1u, ctl, W_BWD_KV_EMPTY)) return;

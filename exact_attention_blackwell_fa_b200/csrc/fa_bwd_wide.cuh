@@ -157,7 +157,7 @@ __device__ void bwd_wide_compute(const BwdParams& p, uint32_t tmem, uint32_t bas
     auto bar = [&](int i) { return bars + 8u * i; };
     const uint64_t sl2x2 = f2pack(p.sl2, p.sl2);
     uint32_t it = 0, unit_it = 0;
-    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+    for (int rnd = 0, ui = walk_unit(0); ui < p.num_units; ui = walk_unit(++rnd)) {
         int win;
         const BwdUnit u = bwd_wide_decode<C::NWIN>(p, ui, win);
         if (!u.keys) continue;  // past the end of its sequence's keys
@@ -278,7 +278,7 @@ __device__ void bwd_wide_dq_reduce(const BwdParams& p, uint32_t tmem, uint32_t b
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     auto bar = [&](int i) { return bars + 8u * i; };
     uint32_t k = 0;  // dQ halves drained so far
-    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+    for (int rnd = 0, ui = walk_unit(0); ui < p.num_units; ui = walk_unit(++rnd)) {
         int win;
         const BwdUnit u = bwd_wide_decode<C::NWIN>(p, ui, win);
         for (int s = 0; s < u.T; ++s) {
@@ -355,7 +355,7 @@ __device__ void bwd_wide_mma(const BwdParams& p, uint32_t tmem, uint32_t base, u
         return I::wait(bar(C::B_DQ_EMPTY), (dq_issued - 1u) & 1u, ctl, W_B256_DQ_EMPTY);
     };
     if constexpr (C::PH == 1) {
-    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+    for (int rnd = 0, ui = walk_unit(0); ui < p.num_units; ui = walk_unit(++rnd)) {
         int win;
         const BwdUnit u = bwd_wide_decode<C::NWIN>(p, ui, win);
         if (u.T == 0) continue;
@@ -410,7 +410,7 @@ __device__ void bwd_wide_mma(const BwdParams& p, uint32_t tmem, uint32_t base, u
     // the unit's own (whose Q, dO and K tiles the transposed products read).  K / V,
     // Q and dO each complete their FULL barrier once per phase.
     uint32_t kv_it = 0, q_it = 0, do_it = 0;
-    for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+    for (int rnd = 0, ui = walk_unit(0); ui < p.num_units; ui = walk_unit(++rnd)) {
         int win;
         const BwdUnit u = bwd_wide_decode<C::NWIN>(p, ui, win);
         if (u.T == 0) continue;
@@ -517,7 +517,7 @@ struct BwdWideLoad {
     }
     __device__ void run(const BwdParams& p)
     {
-        for (int ui = blockIdx.x; ui < p.num_units; ui += gridDim.x) {
+        for (int rnd = 0, ui = walk_unit(0); ui < p.num_units; ui = walk_unit(++rnd)) {
             int win;
             const BwdUnit u = bwd_wide_decode<C::NWIN>(p, ui, win);
             if (u.T == 0) continue;

@@ -36,6 +36,18 @@ struct CtaCtl {
     uint64_t wait_ns;  // limit of a pipeline wait, from the launch parameters
 };
 
+// Unit of round r of a persistent CTA's static walk: rounds take gridDim.x consecutive
+// units, CTA b the b-th of an even round and the b-th from the end of an odd one.
+// With the unit list sorted longest first (causal), a CTA that took a long unit of a
+// round takes a short one of the next, so the CTAs' totals stay level; each round is
+// a permutation of the plain stride's, so every unit below the count is walked once
+// and the first index past the count ends the walk.
+__device__ __forceinline__ int walk_unit(int r)
+{
+    const int g = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+    return r * g + ((r & 1) ? g - 1 - b : b);
+}
+
 __device__ __forceinline__ uint64_t drain_limit(const CtaCtl* ctl)
 {
     return ctl->wait_ns > kWaitTimeoutNs ? ctl->wait_ns : kWaitTimeoutNs;

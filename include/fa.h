@@ -219,17 +219,21 @@ fa_status fa_set_wait_timeout_ms(int ms);
  * Order in which the forward's CTAs take their work units ("[RFC] FA4 --
  * head_dim=256 & head_dim=512", Phase 2 "Persistent + cluster-aware tile
  * scheduler" and Phase 3 short-sequence tuning, CLC scheduling):
- *   FA_SCHED_STATIC (0, the default): a persistent grid of at most one CTA per SM
- *     walks the units with a fixed stride (longest units first under the causal
- *     mask, heads grouped so that concurrent CTAs share K/V in L2);
+ *   FA_SCHED_STATIC (0): a persistent grid of at most one CTA per SM walks the
+ *     units with a fixed stride (longest units first under the causal mask, heads
+ *     grouped so that concurrent CTAs share K/V in L2);
  *   FA_SCHED_CLC (1): when there are more units than SMs, one CTA per unit is
  *     launched and every running CTA takes the next unit by cancelling the launch
- *     of a CTA that has not started (cluster launch control), in unit order.
+ *     of a CTA that has not started (cluster launch control), in unit order;
+ *   FA_SCHED_AUTO (2, the default): CLC for causal launches over at least 4096
+ *     keys (units of unequal length, where taking the next unit when free levels
+ *     the CTAs' work), STATIC otherwise.
  * Process-wide; affects launches made after the call.  Results are identical in
- * both modes.  Any other mode returns FA_ERR_INVALID_ARG.
+ * every mode.  Any other mode returns FA_ERR_INVALID_ARG.
  */
 #define FA_SCHED_STATIC 0
 #define FA_SCHED_CLC 1
+#define FA_SCHED_AUTO 2
 fa_status fa_set_unit_schedule(int mode);
 
 /*

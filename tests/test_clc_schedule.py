@@ -20,15 +20,16 @@ def clc_mode():
     import exact_attention_blackwell_fa_b200 as fa
 
     yield fa
-    fa.fa_set_unit_schedule(fa.FA_SCHED_STATIC)
+    fa.fa_set_unit_schedule(fa.FA_SCHED_AUTO)
 
 
 def test_schedule_mode_arguments():
     from exact_attention_blackwell_fa_b200 import _lib
 
     lib = _lib.load()
-    assert lib.fa_set_unit_schedule(2) == 1 and lib.fa_set_unit_schedule(-1) == 1  # FA_ERR_INVALID_ARG
+    assert lib.fa_set_unit_schedule(3) == 1 and lib.fa_set_unit_schedule(-1) == 1  # FA_ERR_INVALID_ARG
     assert lib.fa_set_unit_schedule(1) == 0 and lib.fa_set_unit_schedule(0) == 0
+    assert lib.fa_set_unit_schedule(2) == 0  # FA_SCHED_AUTO, the default
 
 
 def _both(fa, fn):
