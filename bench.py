@@ -224,12 +224,15 @@ def oracle_cpu_baseline(budget_s=15.0):
 EXTRA_WORKLOADS = [
     dict(B=1, S=16384, H=8, Hkv=8, d=256, causal=False),
     dict(B=2, S=16384, H=16, Hkv=16, d=128, causal=True),
+    dict(B=32, S=1024, H=16, Hkv=16, d=128, causal=True),
 ]
 
 
-def time_extra(fa, make_inputs, Shape, dev, w, steps=5, warmup=3):
+def time_extra(fa, make_inputs, Shape, dev, w, steps=5, warmup=3, min_region_ms=300.0):
     """fa_fwd + fa_bwd on workload w: CUDA events around each call on the launching
-    stream, L2 flushed (a 256 MiB write) before every step; mean per call."""
+    stream, L2 flushed (a 256 MiB write) before every step; mean per call.  Short
+    workloads get more than `steps` timed steps, enough to fill `min_region_ms`, so
+    that the clock sampler (200 ms period) sees the timed region."""
     stream = torch.cuda.current_stream(dev)
     q, k, v, do = make_inputs(Shape(w["B"], w["S"], w["S"], w["H"], w["Hkv"], w["d"]), seed=0, device=dev,
                               with_dout=True)
@@ -238,10 +241,9 @@ def time_extra(fa, make_inputs, Shape, dev, w, steps=5, warmup=3):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(fa.fa_bwd_workspace_size(w["B"], w["S"], w["H"], w["d"]), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-    for i in range(warmup + steps):
+
+    def step(i, e):
         flush.fill_(i & 0xFF)
-        e = ev[i - warmup] if i >= warmup else None
         if e:
             e[0].record(stream)
         fa.fa_fwd(q, k, v, causal=w["causal"], out=o, lse=lse, stream=stream)
@@ -250,6 +252,18 @@ def time_extra(fa, make_inputs, Shape, dev, w, steps=5, warmup=3):
         fa.fa_bwd(q, k, v, o, lse, do, causal=w["causal"], dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
         if e:
             e[2].record(stream)
+
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
+    for i in range(warmup):
+        step(i, None)
+    w1.record(stream)
+    torch.cuda.synchronize(dev)
+    per_step = w0.elapsed_time(w1) / max(warmup, 1)
+    steps = max(steps, min(400, math.ceil(min_region_ms / max(per_step, 1e-3))))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        step(warmup + i, ev[i])
     torch.cuda.synchronize(dev)
     code, detail = fa.fa_last_device_status(stream)
     if code != 0:
